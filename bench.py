@@ -1,0 +1,504 @@
+#!/usr/bin/env python
+"""Throughput of the gated delta rule forward pass on B200, through the C ABI.
+
+One bench "step" is one chunked prefill (the whole prefill path: gates, q/k
+normalisation, intra-chunk UT transform, inter-chunk state passing, outputs and
+final state) over the prefill workload: B=1, T=8192, Hk=Hv=48, dk=dv=128, chunk 32,
+bf16 q/k/v/a/b, fp32 state and fp32 outputs.  ``value`` is prefill tokens/s over all
+ranks.  The decode path is timed beside it on the decode workload (B=64, Hk=Hv=48,
+dk=dv=128, 256 consecutive in-place steps) and reported under ``decode`` as steps/s
+and state GB/s, with its own roofline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 the script runs under torchrun (one process per GPU): every rank runs the
+same per-GPU workload on its own seeded data (weak scaling; the units -- sequences
+x heads -- are independent, so there is no data-path collective), and the timing is
+the max over ranks.  ``--impl reference`` times the fp64 CPU oracle on a bounded
+sample of the same workload (rank 0 only) and prints the same JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDR prefill tokens/s & decode state GB/s (Hv=48, dk=dv=128) vs roofline"
+PREFILL = dict(B=1, T=8192, Hk=48, Hv=48, dk=128, dv=128, chunk=32)
+DECODE = dict(B=64, Hk=48, Hv=48, dk=128, dv=128, steps=256)
+PREFILL_NAME = "chunked prefill B=1 T=8192 Hk=Hv=48 dk=dv=128 chunk=32 (bf16 in, fp32 state/out)"
+DECODE_NAME = "decode B=64 Hk=Hv=48 dk=dv=128, 256 in-place steps (bf16 in, fp32 state/out)"
+
+
+# ----------------------------------------------------------------- algorithmic counts
+
+
+def prefill_alg_bytes(B, T, Hk, Hv, dk, dv, **_):
+    """HBM bytes a prefill must move at least: bf16 q, k, v, a, b in; fp32 o and final
+    state out (zero initial state, nothing read for it)."""
+    tok = B * T
+    return tok * (2 * Hk * dk * 2 + Hv * dv * 2 + 2 * Hv * 2 + Hv * dv * 4) + B * Hv * dk * dv * 4
+
+
+def prefill_alg_flops(B, T, Hk, Hv, dk, dv, chunk, **_):
+    """Flops of the chunked form per token-head: 6 dk dv for W S, Q S and K^T Delta
+    (two flops per MAC) plus ~5 C d for the chunk-local triangles (K K^T, Q K^T, the
+    solve, U, P Delta), each triangle counted once."""
+    d = dk
+    return B * T * Hv * (6 * dk * dv + 5 * chunk * d)
+
+
+def decode_alg_bytes(B, Hk, Hv, dk, dv, **_):
+    """Per step: the fp32 state read and written once, bf16 inputs in, fp32 o out."""
+    return B * Hv * dk * dv * 4 * 2 + B * (2 * Hk * dk * 2 + Hv * dv * 2 + 2 * Hv * 2 +
+                                           Hv * dv * 4)
+
+
+def decode_state_bytes(B, Hv, dk, dv, **_):
+    return B * Hv * dk * dv * 4 * 2
+
+
+# ----------------------------------------------------------------------- environment
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, source="fallback")
+
+
+def kernel_source_hash(name):
+    with open(os.path.join(ROOT, "gated_delta_rule_145_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current source of that kernel (profiles/dram_traffic.txt: file, hash, bytes)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        want = kernel_source_hash(kernel_file)
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel_file \
+                        and parts[1] == want:
+                    return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms in the background; summary of the samples taken
+    inside the marked timed windows."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.samples = []
+        self.windows = []
+        self.proc = None
+        self.gpu_id = gpu_id
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_id)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        def inside(t):
+            return any(a - 0.15 <= t <= b + 0.15 for a, b in self.windows)
+
+        rows = [s for t, s in self.samples if inside(t)] or [s for _, s in self.samples]
+        sm, mx, reasons = [], [], set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(self.REASONS, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
+        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(mx), reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+def gpu_smi_id(dev):
+    import torch
+
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend):
+        if self.world > 1:
+            import torch.distributed as dist
+
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x, device=None):
+        if not self.pg:
+            return x
+        import torch
+
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ------------------------------------------------------------------------ our arm
+
+
+def run_ours(args, dist):
+    import torch
+
+    import gated_delta_rule_145_b200 as gdr
+    from gated_delta_rule_145_b200 import synth
+
+    torch.cuda.set_device(dist.local)
+    dev = torch.device("cuda", dist.local)
+    dist.init("nccl")
+    pk = peaks()
+    sampler = ClockSampler(gpu_smi_id(dist.local))
+    sampler.start()
+
+    # ---- prefill: inputs resident in HBM (seeded per rank)
+    P = PREFILL
+    inp = synth.make_inputs(P["B"], P["T"], P["Hk"], P["Hv"], P["dk"], P["dv"], "bf16",
+                            seed=1002 + 1000 * dist.rank)
+
+    def dev_bf16(x):
+        return torch.from_numpy(x).to(dev).to(torch.bfloat16)
+
+    q, k, v, a, b = (dev_bf16(getattr(inp, n)) for n in ("q", "k", "v", "a", "b"))
+    A_log = torch.from_numpy(inp.A_log).to(dev)
+    dt_bias = torch.from_numpy(inp.dt_bias).to(dev)
+    out = torch.empty((P["B"], P["T"], P["Hv"], P["dv"]), device=dev, dtype=torch.float32)
+    fin = torch.empty((P["B"], P["Hv"], P["dk"], P["dv"]), device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill_once():
+        gdr.gdr_prefill_chunked(q, k, v, a, b, A_log, dt_bias, None, out, fin, None, P["B"],
+                                P["T"], P["Hk"], P["Hv"], P["dk"], P["dv"], P["chunk"],
+                                stream=stream)
+
+    for _ in range(args.warmup):
+        prefill_once()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    region0 = torch.cuda.Event(enable_timing=True)
+    region1 = torch.cuda.Event(enable_timing=True)
+    region0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        prefill_once()
+        ev[i][1].record(stream)
+    region1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    sampler.mark(t_wall0, time.time())
+    region_ms = dist.max(region0.elapsed_time(region1), dev)
+    launch_ms = [s.elapsed_time(e) for s, e in ev]
+    mean_launch_ms = statistics.mean(launch_ms)
+    launches = args.steps  # one kernel per prefill call
+    tokens = P["B"] * P["T"] * args.steps * dist.world
+    value = tokens / (region_ms / 1e3)
+    alg_b = prefill_alg_bytes(**P)
+    alg_f = prefill_alg_flops(**P)
+    achieved_gbs = alg_b / (mean_launch_ms / 1e3) / 1e9
+    traffic = recorded_traffic("chunked_tc.cu")
+
+    # ---- end to end through the public API: pinned host inputs in, outputs back
+    host = {n: torch.from_numpy(getattr(inp, n)).to(torch.bfloat16).pin_memory()
+            for n in ("q", "k", "v", "a", "b")}
+    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    fin_h = torch.empty(fin.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * 4 + fin_h.numel() * 4
+    dbuf = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in host.items()}
+
+    def e2e_once():
+        for n in host:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        gdr.gdr_prefill_chunked(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["a"], dbuf["b"], A_log,
+                                dt_bias, None, out, fin, None, P["B"], P["T"], P["Hk"], P["Hv"],
+                                P["dk"], P["dv"], P["chunk"], stream=stream)
+        out_h.copy_(out, non_blocking=True)
+        fin_h.copy_(fin, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(min(args.warmup, 3)):
+        e2e_once()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    region0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_once()
+    region1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    sampler.mark(t_wall0, time.time())
+    e2e_ms = dist.max(region0.elapsed_time(region1), dev)
+    e2e_value = P["B"] * P["T"] * e2e_steps * dist.world / (e2e_ms / 1e3)
+    del dbuf, host
+
+    # ---- decode: 256 consecutive in-place steps, fresh bf16 inputs per step
+    D = DECODE
+    dinp = synth.make_inputs(D["B"], D["steps"], D["Hk"], D["Hv"], D["dk"], D["dv"], "bf16",
+                             seed=1001 + 1000 * dist.rank, s0_std=0.02)
+
+    def steps_first(x):
+        return torch.from_numpy(np.ascontiguousarray(np.swapaxes(x, 0, 1))).to(dev).to(
+            torch.bfloat16)
+
+    dq, dk_, dv_, da, db = (steps_first(getattr(dinp, n)) for n in ("q", "k", "v", "a", "b"))
+    dA = torch.from_numpy(dinp.A_log).to(dev)
+    ddt = torch.from_numpy(dinp.dt_bias).to(dev)
+    state0 = torch.from_numpy(dinp.init_state).to(dev)
+    state = state0.clone()
+    dout = torch.empty((D["B"], D["Hv"], D["dv"]), device=dev, dtype=torch.float32)
+
+    def decode_pass(events=None):
+        for t in range(D["steps"]):
+            if events is not None:
+                events[t][0].record(stream)
+            gdr.gdr_decode_step(dq[t], dk_[t], dv_[t], da[t], db[t], dA, ddt, state, dout,
+                                D["B"], D["Hk"], D["Hv"], D["dk"], D["dv"], stream=stream)
+            if events is not None:
+                events[t][1].record(stream)
+
+    for _ in range(max(1, args.warmup // 2)):
+        decode_pass()
+    dec_passes = max(1, min(args.steps, 10))
+    dev_events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(D["steps"])] for _ in range(dec_passes)]
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    region0.record(stream)
+    for p_ in range(dec_passes):
+        decode_pass(dev_events[p_])
+    region1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    sampler.mark(t_wall0, time.time())
+    dec_ms = dist.max(region0.elapsed_time(region1), dev)
+    dec_step_ms = [s.elapsed_time(e) for evs in dev_events for s, e in evs]
+    dec_mean_ms = statistics.mean(dec_step_ms)
+    dec_steps_total = dec_passes * D["steps"]
+    dec_value = dec_steps_total / (dec_ms / 1e3)  # per-rank steps/s (each rank steps its batch)
+    dec_state_gbs = decode_state_bytes(**D) * dec_steps_total * dist.world / (dec_ms / 1e3) / 1e9
+    dec_alg = decode_alg_bytes(**D)
+    dec_achieved = dec_alg / (dec_mean_ms / 1e3) / 1e9
+    launches += dec_steps_total
+
+    sampler.stop()
+    clocks = sampler.summary()
+
+    result = None
+    if dist.rank == 0:
+        cpu = None
+        if dist.world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline_sample(inp, seconds_hint=args.cpu_seconds)
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+            "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(region_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 q/k/v/a/b; A_log~U(0,ln16); dt~logU(1e-3,1e-1))",
+            "config": {
+                "workload": PREFILL_NAME, "global_batch": P["B"] * dist.world,
+                "seq_len": P["T"], "heads": P["Hv"], "head_dim": P["dk"], "chunk": P["chunk"],
+                "parallelism": f"dp{dist.world} (independent sequences x heads, no collective)",
+                "l2": "no flush: inputs (302 MB) and outputs (201 MB) exceed the 126 MB L2",
+            },
+            "roofline": {
+                "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved_gbs / pk["hbm_gbs"], 4),
+                "traffic": traffic, "peak_source": pk["source"],
+                "alg_bytes_per_launch": alg_b, "alg_flops_per_launch": alg_f,
+                "kernel_ms": round(mean_launch_ms, 4),
+                "tensor_frac": round(alg_f / (mean_launch_ms / 1e3) / 1e12 / pk["bf16_tflops"], 4),
+            },
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "decode": {
+                "workload": DECODE_NAME, "value": round(dec_value, 1), "unit": "steps/s",
+                "state_gbs": round(dec_state_gbs, 1), "ms_per_step": round(dec_ms / dec_steps_total, 5),
+                "roofline": {"bound": "hbm", "achieved": round(dec_achieved, 1),
+                             "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(dec_achieved / pk["hbm_gbs"], 4),
+                             "traffic": recorded_traffic("recurrent.cu"),
+                             "alg_bytes_per_launch": dec_alg,
+                             "kernel_ms": round(dec_mean_ms, 5)},
+            },
+        }
+    dist.close()
+    return result
+
+
+def cpu_baseline_sample(inp, seconds_hint=15.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the prefill workload: all 48
+    heads over the first T_s tokens (T_s sized from a short probe to take ~seconds_hint)."""
+    from oracle import oracle
+
+    cores = oracle.default_threads()
+
+    def run(Ts):
+        sl = slice(0, Ts)
+        t0 = time.perf_counter()
+        oracle.forward(inp.q[:, sl], inp.k[:, sl], inp.v[:, sl], inp.a[:, sl], inp.b[:, sl],
+                       inp.A_log, inp.dt_bias, nthreads=cores)
+        return time.perf_counter() - t0
+
+    probe = 64
+    t = run(probe)
+    Ts = int(min(inp.q.shape[1], max(probe, probe * seconds_hint / max(t, 1e-3))))
+    t = run(Ts)
+    return {"value": round(Ts / t, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle, all {inp.v.shape[2]} heads, first {Ts} of {inp.q.shape[1]} "
+                      f"tokens of the prefill workload, {t:.1f} s wall"}
+
+
+# ----------------------------------------------------------------- reference arm
+
+
+def run_reference(args, dist):
+    """The oracle timed as the reference arm (rank 0 only; other ranks exit at once)."""
+    if dist.rank != 0:
+        return None
+    from gated_delta_rule_145_b200 import synth
+    from oracle import oracle
+
+    P = PREFILL
+    inp = synth.make_inputs(P["B"], P["T"], P["Hk"], P["Hv"], P["dk"], P["dv"], "bf16", seed=1002)
+    cores = oracle.default_threads()
+    Ts = args.ref_tokens
+    sl = slice(0, Ts)
+    sample = [getattr(inp, n)[:, sl] for n in ("q", "k", "v", "a", "b")]
+
+    def step():
+        oracle.forward(*sample, inp.A_log, inp.dt_bias, nthreads=cores)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = Ts * args.steps / dt
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded recipe)", "impl": "reference",
+        "config": {"workload": PREFILL_NAME, "global_batch": P["B"], "seq_len": P["T"],
+                   "parallelism": "host threads over heads"},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"fp64 oracle, all 48 heads, first {Ts} tokens per step"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-tokens", type=int, default=128,
+                    help="tokens per reference-arm step (all 48 heads)")
+    args = ap.parse_args()
+    dist = Dist()
+    if dist.world != args.gpus:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE={dist.world}; using WORLD_SIZE",
+              file=sys.stderr)
+    res = run_reference(args, dist) if args.impl == "reference" else run_ours(args, dist)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

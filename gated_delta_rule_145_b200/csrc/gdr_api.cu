@@ -1,0 +1,156 @@
+// gdr_api.cu -- the C ABI of libgdr.so (declared in include/gdr.h): argument checks,
+// then kernel launches.  Nothing is enqueued unless every check passes; no call
+// synchronises the stream or allocates device memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdr.h"
+#include "gdr_internal.h"
+
+namespace {
+
+using gdr::FwdParams;
+using gdr::InType;
+
+bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+bool head_size_built(int dk, int dv) { return dk == dv && (dk == 32 || dk == 64 || dk == 128); }
+
+int check_common(const FwdParams& p, int elem_bytes) {
+    // with no tokens the per-token tensors may be empty (NULL); the per-head ones are read
+    if (!p.A_log || !p.dt_bias) return GDR_ERR_NULL;
+    if (p.T > 0 && (!p.q || !p.k || !p.v || !p.a || !p.b || !p.out)) return GDR_ERR_NULL;
+    if (p.nseq < 1 || p.T < 0 || p.Hk < 1 || p.Hv < 1 || p.Hv % p.Hk != 0) return GDR_ERR_SHAPE;
+    if (!head_size_built(p.dk, p.dv)) return GDR_ERR_UNSUPPORTED;
+    if (!aligned(p.q, 16) || !aligned(p.k, 16) || !aligned(p.v, 16) || !aligned(p.out, 16) ||
+        !aligned(p.a, elem_bytes) || !aligned(p.b, elem_bytes) || !aligned(p.A_log, 4) ||
+        !aligned(p.dt_bias, 4) || !aligned(p.init_state, 16) || !aligned(p.final_state, 16) ||
+        !aligned(p.cu_seqlens, 4))
+        return GDR_ERR_ALIGN;
+    // grids are 1-D over (sequence, head[, slice]); keep them within 2^31 - 1
+    if ((long long)p.nseq * p.Hv * 4 > 0x7fffffffLL) return GDR_ERR_SHAPE;
+    return GDR_OK;
+}
+
+int to_status(cudaError_t e) {
+    if (e == cudaSuccess) return GDR_OK;
+    if (e == cudaErrorNotSupported) return GDR_ERR_UNSUPPORTED;
+    return GDR_ERR_CUDA;
+}
+
+FwdParams make_params(const void* q, const void* k, const void* v, const void* a, const void* b,
+                      const float* A_log, const float* dt_bias, const float* init_state,
+                      float* out, float* final_state, const int32_t* cu_seqlens, int B, int T,
+                      int Hk, int Hv, int dk, int dv, int chunk, InType in) {
+    FwdParams p;
+    p.q = q; p.k = k; p.v = v; p.a = a; p.b = b;
+    p.A_log = A_log; p.dt_bias = dt_bias;
+    p.init_state = init_state; p.out = out; p.final_state = final_state;
+    p.cu_seqlens = cu_seqlens;
+    p.nseq = B; p.T = T; p.Hk = Hk; p.Hv = Hv; p.dk = dk; p.dv = dv; p.chunk = chunk;
+    p.in = in;
+    return p;
+}
+
+int prefill_chunked(const FwdParams& p, cudaStream_t stream) {
+    const int rc = check_common(p, p.in == InType::BF16 ? 2 : 4);
+    if (rc != GDR_OK) return rc;
+    if (p.chunk != 32) return GDR_ERR_UNSUPPORTED;
+    if (p.in == InType::BF16 && p.dk == 128 && p.dv == 128) {
+        const cudaError_t e = gdr::launch_chunked_tc(p, stream);
+        if (e != cudaErrorNotSupported) return to_status(e);
+    }
+    return to_status(gdr::launch_chunked_simt(p, stream));
+}
+
+int prefill_recurrent(const FwdParams& p, cudaStream_t stream) {
+    const int rc = check_common(p, p.in == InType::BF16 ? 2 : 4);
+    if (rc != GDR_OK) return rc;
+    return to_status(gdr::launch_recurrent(p, stream));
+}
+
+int decode_step(const void* q, const void* k, const void* v, const void* a, const void* b,
+                const float* A_log, const float* dt_bias, float* state, float* out, int B, int Hk,
+                int Hv, int dk, int dv, InType in, cudaStream_t stream) {
+    if (!state) return GDR_ERR_NULL;
+    // one token per sequence: the dense layout with T = 1, state updated in place
+    const FwdParams p = make_params(q, k, v, a, b, A_log, dt_bias, state, out, state, nullptr, B,
+                                    1, Hk, Hv, dk, dv, 0, in);
+    return prefill_recurrent(p, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdr_prefill_chunked(const void* q, const void* k, const void* v, const void* a,
+                        const void* b, const float* A_log, const float* dt_bias,
+                        const float* init_state, float* out, float* final_state,
+                        const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk, int dv,
+                        int chunk, gdr_stream_t stream) {
+    return prefill_chunked(make_params(q, k, v, a, b, A_log, dt_bias, init_state, out,
+                                       final_state, cu_seqlens, B, T, Hk, Hv, dk, dv, chunk,
+                                       InType::BF16),
+                           (cudaStream_t)stream);
+}
+
+int gdr_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,
+                            const float* b, const float* A_log, const float* dt_bias,
+                            const float* init_state, float* out, float* final_state,
+                            const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                            int dv, int chunk, gdr_stream_t stream) {
+    return prefill_chunked(make_params(q, k, v, a, b, A_log, dt_bias, init_state, out,
+                                       final_state, cu_seqlens, B, T, Hk, Hv, dk, dv, chunk,
+                                       InType::F32),
+                           (cudaStream_t)stream);
+}
+
+int gdr_prefill_recurrent(const void* q, const void* k, const void* v, const void* a,
+                          const void* b, const float* A_log, const float* dt_bias,
+                          const float* init_state, float* out, float* final_state,
+                          const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                          int dv, gdr_stream_t stream) {
+    return prefill_recurrent(make_params(q, k, v, a, b, A_log, dt_bias, init_state, out,
+                                         final_state, cu_seqlens, B, T, Hk, Hv, dk, dv, 0,
+                                         InType::BF16),
+                             (cudaStream_t)stream);
+}
+
+int gdr_prefill_recurrent_f32(const float* q, const float* k, const float* v, const float* a,
+                              const float* b, const float* A_log, const float* dt_bias,
+                              const float* init_state, float* out, float* final_state,
+                              const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                              int dv, gdr_stream_t stream) {
+    return prefill_recurrent(make_params(q, k, v, a, b, A_log, dt_bias, init_state, out,
+                                         final_state, cu_seqlens, B, T, Hk, Hv, dk, dv, 0,
+                                         InType::F32),
+                             (cudaStream_t)stream);
+}
+
+int gdr_decode_step(const void* q, const void* k, const void* v, const void* a, const void* b,
+                    const float* A_log, const float* dt_bias, float* state, float* out, int B,
+                    int Hk, int Hv, int dk, int dv, gdr_stream_t stream) {
+    return decode_step(q, k, v, a, b, A_log, dt_bias, state, out, B, Hk, Hv, dk, dv,
+                       InType::BF16, (cudaStream_t)stream);
+}
+
+int gdr_decode_step_f32(const float* q, const float* k, const float* v, const float* a,
+                        const float* b, const float* A_log, const float* dt_bias, float* state,
+                        float* out, int B, int Hk, int Hv, int dk, int dv, gdr_stream_t stream) {
+    return decode_step(q, k, v, a, b, A_log, dt_bias, state, out, B, Hk, Hv, dk, dv,
+                       InType::F32, (cudaStream_t)stream);
+}
+
+const char* gdr_status_string(int status) {
+    switch (status) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_NULL: return "GDR_ERR_NULL: a required pointer is NULL";
+        case GDR_ERR_SHAPE: return "GDR_ERR_SHAPE: inconsistent sizes";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: head or chunk size not built";
+        case GDR_ERR_ALIGN: return "GDR_ERR_ALIGN: misaligned pointer";
+        case GDR_ERR_CUDA: return "GDR_ERR_CUDA: kernel launch failed";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// gdr_common.cuh -- device helpers shared by the gated delta rule kernels.
+//
+// Gate and normalisation formulas: Mila "GatedDeltaRule.ixx File Reference", Detailed
+// Description (beta = sigmoid(b), g = -exp(A_log) * softplus(a + dt_bias); q and k
+// L2-normalised, q scaled by 1/sqrt(head_key_dim)).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdr {
+
+// Epsilon under the square root of the L2 norm (the pages state none; 1e-6 keeps a
+// zero vector at zero instead of NaN and moves N(0,1) rows by ~1e-8 relative).
+constexpr float kNormEps = 1e-6f;
+
+__device__ __forceinline__ float softplus(float x) {
+    // overflow-free form: max(x, 0) + log1p(exp(-|x|))
+    return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+}
+
+// Log-decay g and write strength beta of one token of one value head.
+__device__ __forceinline__ void gates(float a, float b, float A_log, float dt_bias, float& g,
+                                      float& beta) {
+    g = -expf(A_log) * softplus(a + dt_bias);
+    beta = 1.0f / (1.0f + expf(-b));
+}
+
+__device__ __forceinline__ float inv_norm(float sumsq) { return 1.0f / sqrtf(sumsq + kNormEps); }
+
+// Loads of 4 consecutive input elements (bf16 or fp32) widened to float.
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+    const float2 l = __bfloat1622float2(lo), h = __bfloat1622float2(hi);
+    return make_float4(l.x, l.y, h.x, h.y);
+}
+
+__device__ __forceinline__ float load1(const float* p) { return *p; }
+__device__ __forceinline__ float load1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Token range [t0, t1) of sequence s: packed (cu_seqlens) or dense (s * T).
+__device__ __forceinline__ void seq_range(const int32_t* cu_seqlens, int s, int T, long long& t0,
+                                          long long& t1) {
+    if (cu_seqlens) {
+        t0 = cu_seqlens[s];
+        t1 = cu_seqlens[s + 1];
+    } else {
+        t0 = (long long)s * T;
+        t1 = t0 + T;
+    }
+}
+
+}  // namespace gdr

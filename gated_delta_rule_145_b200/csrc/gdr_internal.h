@@ -1,0 +1,33 @@
+// gdr_internal.h -- launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdr {
+
+enum class InType { BF16, F32 };
+
+// One forward call, already validated by the ABI layer.
+struct FwdParams {
+    const void *q, *k, *v, *a, *b;  // inputs (bf16 or fp32, see `in`)
+    const float *A_log, *dt_bias;   // [Hv]
+    const float* init_state;        // [nseq, Hv, dk, dv] or nullptr
+    float* out;                     // [tokens, Hv, dv]
+    float* final_state;             // [nseq, Hv, dk, dv] or nullptr
+    const int32_t* cu_seqlens;      // [nseq + 1] or nullptr (dense: nseq sequences of T)
+    int nseq, T, Hk, Hv, dk, dv, chunk;
+    InType in;
+};
+
+// Sequential recurrence (decode step and recurrent prefill); recurrent.cu.
+cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
+
+// Chunked prefill on CUDA cores (any supported head size, fp32 or bf16); chunked_simt.cu.
+cudaError_t launch_chunked_simt(const FwdParams& p, cudaStream_t stream);
+
+// Chunked prefill on the tcgen05 tensor cores (bf16, dk = dv = 128, chunk 32);
+// chunked_tc.cu.  Returns cudaErrorNotSupported for shapes it does not handle.
+cudaError_t launch_chunked_tc(const FwdParams& p, cudaStream_t stream);
+
+}  // namespace gdr

@@ -1,0 +1,139 @@
+/*
+ * gdr.h -- C ABI of libgdr.so, the B200 (sm_100a) gated delta rule forward pass.
+ *
+ * The operation (Mila "GatedDeltaRule.ixx File Reference", Detailed Description):
+ * every value head h of every sequence keeps a state S[dk][dv] (fp32, dv contiguous)
+ * and each token t does
+ *     S <- S * exp(g_t)
+ *     delta <- (v_t - k_t^T S) * beta_t
+ *     S <- S + k_t (outer) delta
+ *     o_t <- q_t^T S
+ * with q, k L2-normalised over dk (x / sqrt(sum x^2 + 1e-6)), q further scaled by
+ * 1/sqrt(dk), beta_t = sigmoid(b_t) and g_t = -exp(A_log[h]) * softplus(a_t + dt_bias[h]).
+ * Value head h reads key/query head h / (Hv / Hk) (consecutive grouping).
+ *
+ * Two forms of one definition ("TWO FORMS, ONE DEFINITION" on the same page):
+ *   gdr_prefill_chunked*  -- the chunk-parallel UT-transform form (prefill);
+ *   gdr_decode_step*      -- the sequential recurrence on a persistent state (decode);
+ *   gdr_prefill_recurrent* -- the sequential recurrence over many tokens in one call.
+ * They agree up to floating-point reassociation.  Inference only (no backward).
+ * The "_f32" suffix marks fp32 q, k, v, a, b (tessera PR #77 names its C-ABI symbols
+ * the same way); the unsuffixed calls take bf16 q, k, v, a, b.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device, owned by the
+ *     caller; the library keeps no pointer after the call returns.  Layouts are dense
+ *     row-major with the last dimension contiguous.
+ *   - q, k, v, out, state pointers must be 16-byte aligned; a, b need 4-byte (f32) or
+ *     2-byte (bf16) alignment.
+ *   - A_log and dt_bias are fp32 [Hv].  States are fp32 [Nseq, Hv, dk, dv].  Outputs
+ *     are fp32.
+ *   - `stream` is a cudaStream_t (0 = the legacy default stream).  Calls are
+ *     asynchronous: they enqueue kernels and return; they never synchronise.
+ *   - Every argument is checked before anything is enqueued; on an error nothing is
+ *     launched and the output buffers are untouched.  The calls never throw and never
+ *     abort; they return one of the GDR_* codes below.  GDR_ERR_CUDA reports a launch
+ *     error taken from cudaGetLastError (which clears it).
+ *   - Supported head sizes: dk == dv in {32, 64, 128}; chunk == 32.
+ *   - The library allocates no device memory: all intermediates stay on chip.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* gdr_stream_t; /* cudaStream_t */
+
+#if defined(__GNUC__)
+#define GDR_API __attribute__((visibility("default")))
+#else
+#define GDR_API
+#endif
+
+#define GDR_OK 0
+#define GDR_ERR_NULL (-1)        /* a required pointer is NULL */
+#define GDR_ERR_SHAPE (-2)       /* B, T, Hk, Hv inconsistent (e.g. Hv % Hk != 0) */
+#define GDR_ERR_UNSUPPORTED (-3) /* head size or chunk size not built */
+#define GDR_ERR_ALIGN (-4)       /* a pointer is not aligned as stated above */
+#define GDR_ERR_CUDA (-6)        /* a kernel launch failed */
+
+/*
+ * Chunked (UT-transform) prefill.  Source: Mila "GatedDeltaRule.ixx File Reference",
+ * Detailed Description ("prefill runs the chunked (UT-transform) form ... one
+ * triangular solve per 32 steps"); tessera PR #77 summary, "What landed"
+ * (gated_delta_rule_chunked: the only non-GEMM step is the (I + A)^-1 forward
+ * substitution).
+ *
+ * Dense mode (cu_seqlens == NULL): B sequences of T tokens.
+ *   q, k  [B, T, Hk, dk] bf16      v [B, T, Hv, dv] bf16      a, b [B, T, Hv] bf16
+ *   init_state  [B, Hv, dk, dv] fp32, or NULL for zeros
+ *   out         [B, T, Hv, dv] fp32
+ *   final_state [B, Hv, dk, dv] fp32, or NULL to skip
+ * Varlen mode (cu_seqlens != NULL, device int32 [B + 1], cu_seqlens[0] = 0,
+ * non-decreasing, cu_seqlens[B] = T): B sequences packed along one token axis of
+ * length T; q etc. are [1, T, ...]; states are [B, Hv, dk, dv], one per sequence; each
+ * sequence starts from its own initial state.  Sequences of length 0 are allowed.
+ * init_state may alias final_state.  T == 0 is allowed (the final state is then the
+ * initial state).  chunk must be 32.
+ */
+GDR_API int gdr_prefill_chunked(const void* q, const void* k, const void* v, const void* a,
+                        const void* b, const float* A_log, const float* dt_bias,
+                        const float* init_state, float* out, float* final_state,
+                        const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                        int dv, int chunk, gdr_stream_t stream);
+
+/* As gdr_prefill_chunked with fp32 q, k, v, a, b. */
+GDR_API int gdr_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,
+                            const float* b, const float* A_log, const float* dt_bias,
+                            const float* init_state, float* out, float* final_state,
+                            const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                            int dv, int chunk, gdr_stream_t stream);
+
+/*
+ * One decode step on a persistent state, updated in place.  Source: Mila
+ * "GatedDeltaRule.ixx File Reference", Detailed Description ("Decode runs the
+ * sequential recurrence above").
+ *   q, k  [B, Hk, dk] bf16    v [B, Hv, dv] bf16    a, b [B, Hv] bf16
+ *   state [B, Hv, dk, dv] fp32, read and overwritten with the new state
+ *   out   [B, Hv, dv] fp32
+ */
+GDR_API int gdr_decode_step(const void* q, const void* k, const void* v, const void* a, const void* b,
+                    const float* A_log, const float* dt_bias, float* state, float* out, int B,
+                    int Hk, int Hv, int dk, int dv, gdr_stream_t stream);
+
+/* As gdr_decode_step with fp32 q, k, v, a, b. */
+GDR_API int gdr_decode_step_f32(const float* q, const float* k, const float* v, const float* a,
+                        const float* b, const float* A_log, const float* dt_bias, float* state,
+                        float* out, int B, int Hk, int Hv, int dk, int dv, gdr_stream_t stream);
+
+/*
+ * The sequential recurrence over T tokens in one call (the recurrent form used for
+ * prefill; same arguments and layouts as gdr_prefill_chunked, chunk omitted).  Each
+ * (sequence, head) state stays on chip for the whole sequence.  Source: as
+ * gdr_decode_step; tessera PR #77 summary (gated_delta_rule_recurrent).
+ */
+GDR_API int gdr_prefill_recurrent(const void* q, const void* k, const void* v, const void* a,
+                          const void* b, const float* A_log, const float* dt_bias,
+                          const float* init_state, float* out, float* final_state,
+                          const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                          int dv, gdr_stream_t stream);
+
+/* As gdr_prefill_recurrent with fp32 q, k, v, a, b. */
+GDR_API int gdr_prefill_recurrent_f32(const float* q, const float* k, const float* v, const float* a,
+                              const float* b, const float* A_log, const float* dt_bias,
+                              const float* init_state, float* out, float* final_state,
+                              const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                              int dv, gdr_stream_t stream);
+
+/* A static, human-readable name for a GDR_* status code. */
+GDR_API const char* gdr_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */
