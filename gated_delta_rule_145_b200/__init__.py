@@ -18,7 +18,7 @@ import os
 __all__ = [
     "GdrError", "library", "gdr_prefill_chunked", "gdr_prefill_chunked_f32",
     "gdr_prefill_recurrent", "gdr_prefill_recurrent_f32", "gdr_decode_step",
-    "gdr_decode_step_f32", "gdr_status_string", "prefill", "decode_step", "LIB_PATH",
+    "gdr_decode_step_f32", "gdr_status_string", "gdr_device_status", "prefill", "decode_step", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdr.so")
@@ -29,6 +29,7 @@ GDR_ERR_SHAPE = -2
 GDR_ERR_UNSUPPORTED = -3
 GDR_ERR_ALIGN = -4
 GDR_ERR_CUDA = -6
+GDR_ERR_TIMEOUT = -7
 
 
 class GdrError(RuntimeError):
@@ -63,6 +64,8 @@ def library():
             fn = getattr(lib, name)
             fn.argtypes = args
             fn.restype = _I
+        lib.gdr_device_status.argtypes = [_P]
+        lib.gdr_device_status.restype = _I
         lib.gdr_status_string.argtypes = [_I]
         lib.gdr_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -71,6 +74,11 @@ def library():
 
 def gdr_status_string(status: int) -> str:
     return library().gdr_status_string(int(status)).decode()
+
+
+def gdr_device_status(stream=None) -> int:
+    """Synchronise `stream` and return the device-side status (GDR_OK or an error code)."""
+    return library().gdr_device_status(_stream(stream))
 
 
 def _ptr(x):

@@ -141,6 +141,13 @@ int gdr_decode_step_f32(const float* q, const float* k, const float* v, const fl
                        InType::F32, (cudaStream_t)stream);
 }
 
+int gdr_device_status(gdr_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDR_ERR_CUDA;
+    const int v = gdr::read_and_clear_tc_status();
+    if (v < 0) return GDR_ERR_CUDA;
+    return v ? GDR_ERR_TIMEOUT : GDR_OK;
+}
+
 const char* gdr_status_string(int status) {
     switch (status) {
         case GDR_OK: return "GDR_OK";
@@ -149,6 +156,7 @@ const char* gdr_status_string(int status) {
         case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: head or chunk size not built";
         case GDR_ERR_ALIGN: return "GDR_ERR_ALIGN: misaligned pointer";
         case GDR_ERR_CUDA: return "GDR_ERR_CUDA: kernel launch failed";
+        case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a kernel abandoned a bounded wait";
         default: return "unknown status";
     }
 }

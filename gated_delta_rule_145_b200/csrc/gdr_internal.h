@@ -30,4 +30,8 @@ cudaError_t launch_chunked_simt(const FwdParams& p, cudaStream_t stream);
 // chunked_tc.cu.  Returns cudaErrorNotSupported for shapes it does not handle.
 cudaError_t launch_chunked_tc(const FwdParams& p, cudaStream_t stream);
 
+// Reads and clears the tensor-core kernel's timeout record (1 if set, 0 if not, -1 on a
+// CUDA error); chunked_tc.cu.
+int read_and_clear_tc_status();
+
 }  // namespace gdr

@@ -60,6 +60,7 @@ typedef void* gdr_stream_t; /* cudaStream_t */
 #define GDR_ERR_UNSUPPORTED (-3) /* head size or chunk size not built */
 #define GDR_ERR_ALIGN (-4)       /* a pointer is not aligned as stated above */
 #define GDR_ERR_CUDA (-6)        /* a kernel launch failed */
+#define GDR_ERR_TIMEOUT (-7)     /* a kernel gave up a bounded on-chip wait (see below) */
 
 /*
  * Chunked (UT-transform) prefill.  Source: Mila "GatedDeltaRule.ixx File Reference",
@@ -128,6 +129,15 @@ GDR_API int gdr_prefill_recurrent_f32(const float* q, const float* k, const floa
                               const float* init_state, float* out, float* final_state,
                               const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
                               int dv, gdr_stream_t stream);
+
+/*
+ * Device-side status of the kernels enqueued so far.  Synchronises `stream`, then returns
+ * GDR_ERR_TIMEOUT if any tensor-core prefill kernel abandoned one of its bounded waits
+ * (each wait on an mbarrier gives up after 2 s, records the event and lets the kernel
+ * exit instead of hanging), GDR_ERR_CUDA if the stream reports an error, else GDR_OK.
+ * The timeout record is cleared by the call.
+ */
+GDR_API int gdr_device_status(gdr_stream_t stream);
 
 /* A static, human-readable name for a GDR_* status code. */
 GDR_API const char* gdr_status_string(int status);
