@@ -220,6 +220,121 @@ class Dist:
 # ------------------------------------------------------------------------ our arm
 
 
+def _timed(dist, dev, stream, sampler, fn, n):
+    """Run fn() n times between a barrier + synchronize on both sides; returns the max
+    over ranks of the device time (ms) measured with CUDA events on `stream`."""
+    import torch
+
+    r0 = torch.cuda.Event(enable_timing=True)
+    r1 = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    r0.record(stream)
+    for i in range(n):
+        fn(i)
+    r1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    sampler.mark(t_wall0, time.time())
+    return dist.max(r0.elapsed_time(r1), dev)
+
+
+def bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth):
+    import torch
+
+    inp = synth.make_inputs(P["B"], P["T"], P["Hk"], P["Hv"], P["dk"], P["dv"], "bf16",
+                            seed=1002 + 1000 * dist.rank)
+
+    def dev_bf16(x):
+        return torch.from_numpy(x).to(dev).to(torch.bfloat16)
+
+    q, k, v, a, b = (dev_bf16(getattr(inp, n)) for n in ("q", "k", "v", "a", "b"))
+    A_log = torch.from_numpy(inp.A_log).to(dev)
+    dt_bias = torch.from_numpy(inp.dt_bias).to(dev)
+    out = torch.empty((P["B"], P["T"], P["Hv"], P["dv"]), device=dev, dtype=torch.float32)
+    fin = torch.empty((P["B"], P["Hv"], P["dk"], P["dv"]), device=dev, dtype=torch.float32)
+
+    def launch(qq, kk, vv, aa, bb):
+        gdr.gdr_prefill_chunked(qq, kk, vv, aa, bb, A_log, dt_bias, None, out, fin, None,
+                                P["B"], P["T"], P["Hk"], P["Hv"], P["dk"], P["dv"], P["chunk"],
+                                stream=stream)
+
+    for _ in range(args.warmup):
+        launch(q, k, v, a, b)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+
+    def step(i):
+        ev[i][0].record(stream)
+        launch(q, k, v, a, b)
+        ev[i][1].record(stream)
+
+    region_ms = _timed(dist, dev, stream, sampler, step, args.steps)
+    res = dict(inp=inp, region_ms=region_ms, launches=args.steps,
+               kernel_ms=statistics.mean(s.elapsed_time(e) for s, e in ev))
+    if args.no_e2e:
+        return res
+    # ---- end to end through the public API: pinned host inputs in, outputs back
+    host = {n: torch.from_numpy(getattr(inp, n)).to(torch.bfloat16).pin_memory()
+            for n in ("q", "k", "v", "a", "b")}
+    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    fin_h = torch.empty(fin.shape, dtype=torch.float32).pin_memory()
+    dbuf = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in host.items()}
+
+    def e2e(_i):
+        for n in host:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        launch(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["a"], dbuf["b"])
+        out_h.copy_(out, non_blocking=True)
+        fin_h.copy_(fin, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for i in range(min(args.warmup, 3)):
+        e2e(i)
+    e2e_ms = _timed(dist, dev, stream, sampler, e2e, e2e_steps)
+    res.update(e2e_steps=e2e_steps, e2e_ms=e2e_ms, launches=args.steps + e2e_steps,
+               h2d=sum(t.numel() * t.element_size() for t in host.values()),
+               d2h=out_h.numel() * 4 + fin_h.numel() * 4)
+    return res
+
+
+def bench_decode(args, dist, dev, stream, sampler, gdr, synth):
+    import torch
+
+    D = DECODE
+    dinp = synth.make_inputs(D["B"], D["steps"], D["Hk"], D["Hv"], D["dk"], D["dv"], "bf16",
+                             seed=1001 + 1000 * dist.rank, s0_std=0.02)
+
+    def steps_first(x):
+        return torch.from_numpy(np.ascontiguousarray(np.swapaxes(x, 0, 1))).to(dev).to(
+            torch.bfloat16)
+
+    dq, dk_, dv_, da, db = (steps_first(getattr(dinp, n)) for n in ("q", "k", "v", "a", "b"))
+    dA = torch.from_numpy(dinp.A_log).to(dev)
+    ddt = torch.from_numpy(dinp.dt_bias).to(dev)
+    state = torch.from_numpy(dinp.init_state).to(dev)
+    dout = torch.empty((D["B"], D["Hv"], D["dv"]), device=dev, dtype=torch.float32)
+    passes = max(1, min(args.steps, 10))
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(D["steps"])] for _ in range(passes)]
+
+    def one_pass(pi, record=True):
+        for t in range(D["steps"]):
+            if record:
+                ev[pi][t][0].record(stream)
+            gdr.gdr_decode_step(dq[t], dk_[t], dv_[t], da[t], db[t], dA, ddt, state, dout,
+                                D["B"], D["Hk"], D["Hv"], D["dk"], D["dv"], stream=stream)
+            if record:
+                ev[pi][t][1].record(stream)
+
+    for _ in range(max(1, args.warmup // 2)):
+        one_pass(0, record=False)
+    ms = _timed(dist, dev, stream, sampler, one_pass, passes)
+    return dict(ms=ms, steps=passes * D["steps"],
+                kernel_ms=statistics.mean(s.elapsed_time(e) for evs in ev for s, e in evs))
+
+
 def run_ours(args, dist):
     import torch
 
@@ -232,185 +347,77 @@ def run_ours(args, dist):
     pk = peaks()
     sampler = ClockSampler(gpu_smi_id(dist.local))
     sampler.start()
-
-    # ---- prefill: inputs resident in HBM (seeded per rank)
-    P = PREFILL
-    inp = synth.make_inputs(P["B"], P["T"], P["Hk"], P["Hv"], P["dk"], P["dv"], "bf16",
-                            seed=1002 + 1000 * dist.rank)
-
-    def dev_bf16(x):
-        return torch.from_numpy(x).to(dev).to(torch.bfloat16)
-
-    q, k, v, a, b = (dev_bf16(getattr(inp, n)) for n in ("q", "k", "v", "a", "b"))
-    A_log = torch.from_numpy(inp.A_log).to(dev)
-    dt_bias = torch.from_numpy(inp.dt_bias).to(dev)
-    out = torch.empty((P["B"], P["T"], P["Hv"], P["dv"]), device=dev, dtype=torch.float32)
-    fin = torch.empty((P["B"], P["Hv"], P["dk"], P["dv"]), device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
-
-    def prefill_once():
-        gdr.gdr_prefill_chunked(q, k, v, a, b, A_log, dt_bias, None, out, fin, None, P["B"],
-                                P["T"], P["Hk"], P["Hv"], P["dk"], P["dv"], P["chunk"],
-                                stream=stream)
-
-    for _ in range(args.warmup):
-        prefill_once()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    dist.barrier()
-    torch.cuda.synchronize(dev)
-    t_wall0 = time.time()
-    region0 = torch.cuda.Event(enable_timing=True)
-    region1 = torch.cuda.Event(enable_timing=True)
-    region0.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        prefill_once()
-        ev[i][1].record(stream)
-    region1.record(stream)
-    torch.cuda.synchronize(dev)
-    dist.barrier()
-    sampler.mark(t_wall0, time.time())
-    region_ms = dist.max(region0.elapsed_time(region1), dev)
-    launch_ms = [s.elapsed_time(e) for s, e in ev]
-    mean_launch_ms = statistics.mean(launch_ms)
-    launches = args.steps  # one kernel per prefill call
-    tokens = P["B"] * P["T"] * args.steps * dist.world
-    value = tokens / (region_ms / 1e3)
-    alg_b = prefill_alg_bytes(**P)
-    alg_f = prefill_alg_flops(**P)
-    achieved_gbs = alg_b / (mean_launch_ms / 1e3) / 1e9
-    traffic = recorded_traffic("chunked_tc.cu")
-
-    # ---- end to end through the public API: pinned host inputs in, outputs back
-    host = {n: torch.from_numpy(getattr(inp, n)).to(torch.bfloat16).pin_memory()
-            for n in ("q", "k", "v", "a", "b")}
-    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    fin_h = torch.empty(fin.shape, dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * 4 + fin_h.numel() * 4
-    dbuf = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in host.items()}
-
-    def e2e_once():
-        for n in host:
-            dbuf[n].copy_(host[n], non_blocking=True)
-        gdr.gdr_prefill_chunked(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["a"], dbuf["b"], A_log,
-                                dt_bias, None, out, fin, None, P["B"], P["T"], P["Hk"], P["Hv"],
-                                P["dk"], P["dv"], P["chunk"], stream=stream)
-        out_h.copy_(out, non_blocking=True)
-        fin_h.copy_(fin, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(min(args.warmup, 3)):
-        e2e_once()
-    dist.barrier()
-    torch.cuda.synchronize(dev)
-    t_wall0 = time.time()
-    region0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_once()
-    region1.record(stream)
-    torch.cuda.synchronize(dev)
-    dist.barrier()
-    sampler.mark(t_wall0, time.time())
-    e2e_ms = dist.max(region0.elapsed_time(region1), dev)
-    e2e_value = P["B"] * P["T"] * e2e_steps * dist.world / (e2e_ms / 1e3)
-    del dbuf, host
-
-    # ---- decode: 256 consecutive in-place steps, fresh bf16 inputs per step
-    D = DECODE
-    dinp = synth.make_inputs(D["B"], D["steps"], D["Hk"], D["Hv"], D["dk"], D["dv"], "bf16",
-                             seed=1001 + 1000 * dist.rank, s0_std=0.02)
-
-    def steps_first(x):
-        return torch.from_numpy(np.ascontiguousarray(np.swapaxes(x, 0, 1))).to(dev).to(
-            torch.bfloat16)
-
-    dq, dk_, dv_, da, db = (steps_first(getattr(dinp, n)) for n in ("q", "k", "v", "a", "b"))
-    dA = torch.from_numpy(dinp.A_log).to(dev)
-    ddt = torch.from_numpy(dinp.dt_bias).to(dev)
-    state0 = torch.from_numpy(dinp.init_state).to(dev)
-    state = state0.clone()
-    dout = torch.empty((D["B"], D["Hv"], D["dv"]), device=dev, dtype=torch.float32)
-
-    def decode_pass(events=None):
-        for t in range(D["steps"]):
-            if events is not None:
-                events[t][0].record(stream)
-            gdr.gdr_decode_step(dq[t], dk_[t], dv_[t], da[t], db[t], dA, ddt, state, dout,
-                                D["B"], D["Hk"], D["Hv"], D["dk"], D["dv"], stream=stream)
-            if events is not None:
-                events[t][1].record(stream)
-
-    for _ in range(max(1, args.warmup // 2)):
-        decode_pass()
-    dec_passes = max(1, min(args.steps, 10))
-    dev_events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(D["steps"])] for _ in range(dec_passes)]
-    dist.barrier()
-    torch.cuda.synchronize(dev)
-    t_wall0 = time.time()
-    region0.record(stream)
-    for p_ in range(dec_passes):
-        decode_pass(dev_events[p_])
-    region1.record(stream)
-    torch.cuda.synchronize(dev)
-    dist.barrier()
-    sampler.mark(t_wall0, time.time())
-    dec_ms = dist.max(region0.elapsed_time(region1), dev)
-    dec_step_ms = [s.elapsed_time(e) for evs in dev_events for s, e in evs]
-    dec_mean_ms = statistics.mean(dec_step_ms)
-    dec_steps_total = dec_passes * D["steps"]
-    dec_value = dec_steps_total / (dec_ms / 1e3)  # per-rank steps/s (each rank steps its batch)
-    dec_state_gbs = decode_state_bytes(**D) * dec_steps_total * dist.world / (dec_ms / 1e3) / 1e9
-    dec_alg = decode_alg_bytes(**D)
-    dec_achieved = dec_alg / (dec_mean_ms / 1e3) / 1e9
-    launches += dec_steps_total
-
+    P = dict(PREFILL)
+    if args.T:
+        P["T"] = args.T
+    pre = dec = None
+    if args.only in (None, "prefill"):
+        pre = bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth)
+    if args.only in (None, "decode"):
+        dec = bench_decode(args, dist, dev, stream, sampler, gdr, synth)
     sampler.stop()
     clocks = sampler.summary()
 
     result = None
     if dist.rank == 0:
-        cpu = None
-        if dist.world == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline_sample(inp, seconds_hint=args.cpu_seconds)
-        result = {
-            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
-            "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(region_ms / args.steps, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) bf16 q/k/v/a/b; A_log~U(0,ln16); dt~logU(1e-3,1e-1))",
-            "config": {
-                "workload": PREFILL_NAME, "global_batch": P["B"] * dist.world,
-                "seq_len": P["T"], "heads": P["Hv"], "head_dim": P["dk"], "chunk": P["chunk"],
-                "parallelism": f"dp{dist.world} (independent sequences x heads, no collective)",
-                "l2": "no flush: inputs (302 MB) and outputs (201 MB) exceed the 126 MB L2",
-            },
-            "roofline": {
-                "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved_gbs / pk["hbm_gbs"], 4),
-                "traffic": traffic, "peak_source": pk["source"],
-                "alg_bytes_per_launch": alg_b, "alg_flops_per_launch": alg_f,
-                "kernel_ms": round(mean_launch_ms, 4),
-                "tensor_frac": round(alg_f / (mean_launch_ms / 1e3) / 1e12 / pk["bf16_tflops"], 4),
-            },
-            "cpu_baseline": cpu,
-            "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "gpu_launches": launches,
-            "clocks": clocks,
-            "decode": {
-                "workload": DECODE_NAME, "value": round(dec_value, 1), "unit": "steps/s",
-                "state_gbs": round(dec_state_gbs, 1), "ms_per_step": round(dec_ms / dec_steps_total, 5),
-                "roofline": {"bound": "hbm", "achieved": round(dec_achieved, 1),
-                             "peak": pk["hbm_gbs"], "unit": "GB/s",
-                             "frac": round(dec_achieved / pk["hbm_gbs"], 4),
+        result = {"metric": METRIC, "n_gpus": dist.world, "steps": args.steps,
+                  "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                  "vs_baseline": None, "dtype": "bf16",
+                  "data": "synthetic (seeded N(0,1) bf16 q/k/v/a/b; A_log~U(0,ln16); "
+                          "dt~logU(1e-3,1e-1))", "clocks": clocks, "gpu_launches": 0}
+        if pre is not None:
+            alg_b, alg_f = prefill_alg_bytes(**P), prefill_alg_flops(**P)
+            achieved = alg_b / (pre["kernel_ms"] / 1e3) / 1e9
+            cpu = None
+            if dist.world == 1 and not args.no_cpu_baseline and args.only is None:
+                cpu = cpu_baseline_sample(pre["inp"], seconds_hint=args.cpu_seconds)
+            result.update({
+                "value": round(P["B"] * P["T"] * args.steps * dist.world /
+                               (pre["region_ms"] / 1e3), 1),
+                "unit": "tokens/s", "ms_per_step": round(pre["region_ms"] / args.steps, 4),
+                "config": {
+                    "workload": PREFILL_NAME if P["T"] == PREFILL["T"] else
+                    PREFILL_NAME.replace("T=8192", f"T={P['T']}"),
+                    "global_batch": P["B"] * dist.world, "seq_len": P["T"],
+                    "heads": P["Hv"], "head_dim": P["dk"], "chunk": P["chunk"],
+                    "parallelism": f"dp{dist.world} (independent sequences x heads, "
+                                   "no collective)",
+                    "l2": "no flush: inputs (302 MB) and outputs (201 MB) exceed the 126 MB L2",
+                },
+                "roofline": {
+                    "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                    "traffic": recorded_traffic("chunked_tc.cu"), "peak_source": pk["source"],
+                    "alg_bytes_per_launch": alg_b, "alg_flops_per_launch": alg_f,
+                    "kernel_ms": round(pre["kernel_ms"], 4),
+                    "tensor_frac": round(alg_f / (pre["kernel_ms"] / 1e3) / 1e12 /
+                                         pk["bf16_tflops"], 4),
+                },
+                "cpu_baseline": cpu,
+            })
+            result["gpu_launches"] += pre["launches"]
+            if "e2e_ms" in pre:
+                result["e2e"] = {"value": round(P["B"] * P["T"] * pre["e2e_steps"] * dist.world /
+                                                (pre["e2e_ms"] / 1e3), 1),
+                                 "unit": "tokens/s", "h2d_bytes_per_step": pre["h2d"],
+                                 "d2h_bytes_per_step": pre["d2h"], "steps": pre["e2e_steps"]}
+        if dec is not None:
+            D = DECODE
+            dalg = decode_alg_bytes(**D)
+            dach = dalg / (dec["kernel_ms"] / 1e3) / 1e9
+            result["decode"] = {
+                "workload": DECODE_NAME, "value": round(dec["steps"] / (dec["ms"] / 1e3), 1),
+                "unit": "steps/s",
+                "state_gbs": round(decode_state_bytes(**D) * dec["steps"] * dist.world /
+                                   (dec["ms"] / 1e3) / 1e9, 1),
+                "ms_per_step": round(dec["ms"] / dec["steps"], 5),
+                "roofline": {"bound": "hbm", "achieved": round(dach, 1), "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(dach / pk["hbm_gbs"], 4),
                              "traffic": recorded_traffic("recurrent.cu"),
-                             "alg_bytes_per_launch": dec_alg,
-                             "kernel_ms": round(dec_mean_ms, 5)},
-            },
-        }
+                             "alg_bytes_per_launch": dalg,
+                             "kernel_ms": round(dec["kernel_ms"], 5)}}
+            result["gpu_launches"] += dec["steps"]
     dist.close()
     return result
 
@@ -490,6 +497,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=128,
                     help="tokens per reference-arm step (all 48 heads)")
+    ap.add_argument("--only", choices=("prefill", "decode"), default=None,
+                    help="time one path only (profiling runs; not the contract line)")
+    ap.add_argument("--T", type=int, default=0, help="prefill length override (profiling)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     args = ap.parse_args()
     dist = Dist()
     if dist.world != args.gpus:
