@@ -271,7 +271,8 @@ def bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth):
         ev[i][1].record(stream)
 
     region_ms = _timed(dist, dev, stream, sampler, step, args.steps)
-    res = dict(inp=inp, region_ms=region_ms, launches=args.steps,
+    # two kernels per call: intra-chunk, then state passing
+    res = dict(inp=inp, region_ms=region_ms, launches=2 * args.steps,
                kernel_ms=statistics.mean(s.elapsed_time(e) for s, e in ev))
     if args.no_e2e:
         return res
@@ -293,7 +294,7 @@ def bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth):
     for i in range(min(args.warmup, 3)):
         e2e(i)
     e2e_ms = _timed(dist, dev, stream, sampler, e2e, e2e_steps)
-    res.update(e2e_steps=e2e_steps, e2e_ms=e2e_ms, launches=args.steps + e2e_steps,
+    res.update(e2e_steps=e2e_steps, e2e_ms=e2e_ms, launches=2 * (args.steps + e2e_steps),
                h2d=sum(t.numel() * t.element_size() for t in host.values()),
                d2h=out_h.numel() * 4 + fin_h.numel() * 4)
     return res
@@ -388,7 +389,7 @@ def run_ours(args, dist):
                 "roofline": {
                     "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                    "traffic": recorded_traffic("chunked_tc.cu"), "peak_source": pk["source"],
+                    "traffic": recorded_traffic("prefill_tc.cu"), "peak_source": pk["source"],
                     "alg_bytes_per_launch": alg_b, "alg_flops_per_launch": alg_f,
                     "kernel_ms": round(pre["kernel_ms"], 4),
                     "tensor_frac": round(alg_f / (pre["kernel_ms"] / 1e3) / 1e12 /

@@ -28,6 +28,7 @@ GDR_ERR_NULL = -1
 GDR_ERR_SHAPE = -2
 GDR_ERR_UNSUPPORTED = -3
 GDR_ERR_ALIGN = -4
+GDR_ERR_OOM = -5
 GDR_ERR_CUDA = -6
 GDR_ERR_TIMEOUT = -7
 
@@ -68,6 +69,8 @@ def library():
         lib.gdr_device_status.restype = _I
         lib.gdr_status_string.argtypes = [_I]
         lib.gdr_status_string.restype = ctypes.c_char_p
+        lib.gdr_release_workspace.argtypes = []
+        lib.gdr_release_workspace.restype = None
         _lib = lib
     return _lib
 
@@ -79,6 +82,11 @@ def gdr_status_string(status: int) -> str:
 def gdr_device_status(stream=None) -> int:
     """Synchronise `stream` and return the device-side status (GDR_OK or an error code)."""
     return library().gdr_device_status(_stream(stream))
+
+
+def gdr_release_workspace() -> None:
+    """Return the workspace memory cached by earlier chunked prefill calls."""
+    library().gdr_release_workspace()
 
 
 def _ptr(x):

@@ -1,6 +1,7 @@
 // gdr_api.cu -- the C ABI of libgdr.so (declared in include/gdr.h): argument checks,
 // then kernel launches.  Nothing is enqueued unless every check passes; no call
-// synchronises the stream or allocates device memory.
+// synchronises the stream.  The tensor-core prefill takes its workspace from a private
+// stream-ordered pool (prefill_tc.cu).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,6 +36,7 @@ int check_common(const FwdParams& p, int elem_bytes) {
 int to_status(cudaError_t e) {
     if (e == cudaSuccess) return GDR_OK;
     if (e == cudaErrorNotSupported) return GDR_ERR_UNSUPPORTED;
+    if (e == cudaErrorMemoryAllocation) return GDR_ERR_OOM;
     return GDR_ERR_CUDA;
 }
 
@@ -57,7 +59,7 @@ int prefill_chunked(const FwdParams& p, cudaStream_t stream) {
     if (rc != GDR_OK) return rc;
     if (p.chunk != 32) return GDR_ERR_UNSUPPORTED;
     if (p.in == InType::BF16 && p.dk == 128 && p.dv == 128) {
-        const cudaError_t e = gdr::launch_chunked_tc(p, stream);
+        const cudaError_t e = gdr::launch_prefill_tc(p, stream);
         if (e != cudaErrorNotSupported) return to_status(e);
     }
     return to_status(gdr::launch_chunked_simt(p, stream));
@@ -148,6 +150,8 @@ int gdr_device_status(gdr_stream_t stream) {
     return v ? GDR_ERR_TIMEOUT : GDR_OK;
 }
 
+void gdr_release_workspace(void) { gdr::workspace_release(); }
+
 const char* gdr_status_string(int status) {
     switch (status) {
         case GDR_OK: return "GDR_OK";
@@ -155,6 +159,7 @@ const char* gdr_status_string(int status) {
         case GDR_ERR_SHAPE: return "GDR_ERR_SHAPE: inconsistent sizes";
         case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: head or chunk size not built";
         case GDR_ERR_ALIGN: return "GDR_ERR_ALIGN: misaligned pointer";
+        case GDR_ERR_OOM: return "GDR_ERR_OOM: the prefill workspace could not be allocated";
         case GDR_ERR_CUDA: return "GDR_ERR_CUDA: kernel launch failed";
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a kernel abandoned a bounded wait";
         default: return "unknown status";

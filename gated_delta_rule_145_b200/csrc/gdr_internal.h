@@ -26,12 +26,22 @@ cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
 // Chunked prefill on CUDA cores (any supported head size, fp32 or bf16); chunked_simt.cu.
 cudaError_t launch_chunked_simt(const FwdParams& p, cudaStream_t stream);
 
-// Chunked prefill on the tcgen05 tensor cores (bf16, dk = dv = 128, chunk 32);
-// chunked_tc.cu.  Returns cudaErrorNotSupported for shapes it does not handle.
-cudaError_t launch_chunked_tc(const FwdParams& p, cudaStream_t stream);
+// Chunked prefill on the tcgen05 tensor cores (bf16, dk = dv = 128, chunk 32):
+// the intra-chunk kernel, then the state-passing kernel, with a workspace of one record
+// per (chunk, value head) taken from the library's stream-ordered pool; prefill_tc.cu.
+// Returns cudaErrorNotSupported for shapes it does not handle.
+cudaError_t launch_prefill_tc(const FwdParams& p, cudaStream_t stream);
 
-// Reads and clears the tensor-core kernel's timeout record (1 if set, 0 if not, -1 on a
-// CUDA error); chunked_tc.cu.
+// Bytes of workspace the tensor-core prefill needs for `p`, and the launch on a caller's
+// workspace of at least that size (16-byte aligned); prefill_tc.cu.
+size_t prefill_tc_workspace_bytes(const FwdParams& p);
+cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stream);
+
+// Returns the cached workspace memory of every device to the system; prefill_tc.cu.
+void workspace_release();
+
+// Reads and clears the tensor-core kernels' timeout record (nonzero if set, 0 if not,
+// -1 on a CUDA error); prefill_tc.cu.
 int read_and_clear_tc_status();
 
 }  // namespace gdr

@@ -1,0 +1,1034 @@
+// prefill_tc.cu -- chunked (UT-transform) prefill of the gated delta rule on the sm_100a
+// tensor cores (tcgen05 with accumulators in tensor memory, operands fed by TMA).
+//
+// Sources: Mila "GatedDeltaRule.ixx File Reference", Detailed Description (the step, the
+// gates, the normalisation; prefill runs the chunked UT-transform form with one
+// triangular solve per 32 steps); tessera PR #77 summary, "What landed" (the chunked
+// form's only non-GEMM step is the (I + A)^-1 forward substitution).
+//
+// Algebra.  Chunk c holds C = 32 tokens; S_c is the state at its start; K_c, Q_c, V_c are
+// the raw bf16 rows; r_k, r_q the inverse row norms (r_q including 1/sqrt(dk)); G the
+// in-chunk cumulative log-decay (G_i = g_1 + ... + g_i); gamma_c = e^{G_C}.
+//   A[i,j] = beta_i e^{G_i-G_j} r_k,i r_k,j (K K^T)[i,j]  (j < i)      T = (I + A)^-1
+//   Wt = T diag(beta e^G r_k)    Tb = T diag(beta)
+//   P[i,j] = e^{G_i-G_j} r_q,i r_k,j (Q K^T)[i,j]          (j <= i)
+//   E = e^G r_q                  D = e^{G_C - G} r_k
+//   Delta_c = Tb V_c - Wt K_c S_c
+//   O_c     = diag(E) Q_c S_c + P Delta_c
+//   S_{c+1} = gamma_c S_c + K_c^T diag(D) Delta_c
+// One chunk of lookahead takes the state out of the critical chain: since
+//   K_{c+1} S_{c+1} = gamma_c K_{c+1} S_c + K_{c+1} K_c^T diag(D_c) Delta_c,
+//   Delta_{c+1} = Tb_{c+1} V_{c+1} - Wt_{c+1} Y_{c+1} - M_{c+1} Delta_c   with
+//   Y_{c+1} = gamma_c K_{c+1} S_c,   M_{c+1} = Wt_{c+1} K_{c+1} K_c^T diag(D_c).
+// Delta_{c+1} follows from Delta_c through one 32-deep product; the state enters only
+// through Y_{c+1}, which needs S_c, a chunk earlier.
+//
+// Precision.  Every tensor-core product has a raw bf16 input (exact) on one side or splits
+// an fp32 operand into bf16 hi + lo (about 16 significant bits); derived x derived
+// products take hi*hi + hi*lo + lo*hi.  Accumulation is fp32.  Decay factors are exp of
+// non-positive numbers.
+//
+// Kernels:
+//   intra_chunk_kernel  one CTA per (chunk, value head), all independent.  Gates, norms,
+//                       the Gram block [K;Q] [K_prev;K]^T on tcgen05, A and P, the forward
+//                       substitution T [diag(w) | diag(beta) | diag(w) K K_prev^T diag(D_prev)]
+//                       = [Wt | Tb | M] with one thread per right-hand-side column, and a
+//                       record of the chunk's operands (chunk_record.h) in the workspace.
+//   state_pass_kernel   one CTA per (sequence, value head, 48-column slice of dv); the
+//                       slice's state stays in registers for the whole sequence.
+#include <mutex>
+
+#include "chunk_record.h"
+#include "gdr_common.cuh"
+#include "gdr_internal.h"
+#include "tcgen05.cuh"
+#include "tma_map.h"
+
+namespace gdr {
+
+// Set when a bounded wait inside a kernel expired (read by gdr_device_status()).
+__device__ int g_tc_status = 0;
+
+#ifdef GDR_TC_STAMP
+// Cycle stamps of CTA 0 of the state-passing kernel, steps 0-63 (debug builds only).
+__device__ long long* g_stamp = nullptr;
+#define STAMP(b, k)                                                                       \
+    do {                                                                                  \
+        if (stamp_ptr && (b) >= 0 && (b) < 64 && (threadIdx.x & 31) == 0)                 \
+            stamp_ptr[(b) * 32 + (k)] = clock64();                                        \
+    } while (0)
+#define STAMP_INIT long long* stamp_ptr = blockIdx.x == 0 ? g_stamp : nullptr
+#else
+#define STAMP(b, k)
+#define STAMP_INIT
+#endif
+
+namespace {
+
+using namespace tc;
+using rec::C;
+using rec::DK;
+using rec::DV;
+using rec::IMG;
+
+// Gates with the fast exponential/logarithm (relative error ~1e-7, far inside the
+// tolerance).  exp(A_log) is hoisted by the caller.
+__device__ __forceinline__ void gates_fast(float a, float b, float eA, float dt_bias, float& g,
+                                           float& beta) {
+    const float x = a + dt_bias;
+    g = -eA * (fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x))));
+    beta = __frcp_rn(1.f + __expf(-b));
+}
+
+__device__ __forceinline__ float inv_norm_fast(float sumsq) { return rsqrtf(sumsq + kNormEps); }
+
+__device__ __forceinline__ float warp_inclusive_scan(float x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    return x;
+}
+
+// TMEM lane field of the 32 lanes warp `warp` may access.
+__device__ __forceinline__ uint32_t lane_base(int warp) {
+    return (uint32_t)((warp & 3) * 32) << 16;
+}
+
+// A descriptor moved by `bytes` (the start address field holds address >> 4).
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// Sum of squares of the 64 bf16 values in 128 bytes of shared memory.
+__device__ __forceinline__ float sumsq64(const uint8_t* line) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint4 u = *reinterpret_cast<const uint4*>(line + 16 * j);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            s0 += f.x * f.x;
+            s1 += f.y * f.y;
+        }
+    }
+    return s0 + s1;
+}
+
+// Row m of a 32 x 32 operand image (hi and lo parts): sgn * src[0..31].
+__device__ __forceinline__ void store_image_row(const float* __restrict__ src, float sgn,
+                                                uint8_t* hi, uint8_t* lo, int m) {
+#pragma unroll
+    for (int kc = 0; kc < 4; ++kc) {
+        const float4 s0 = *reinterpret_cast<const float4*>(src + 8 * kc);
+        const float4 s1 = *reinterpret_cast<const float4*>(src + 8 * kc + 4);
+        uint4 hv, lv;
+        split2(sgn * s0.x, sgn * s0.y, hv.x, lv.x);
+        split2(sgn * s0.z, sgn * s0.w, hv.y, lv.y);
+        split2(sgn * s1.x, sgn * s1.y, hv.z, lv.z);
+        split2(sgn * s1.z, sgn * s1.w, hv.w, lv.w);
+        *reinterpret_cast<uint4*>(hi + rec::k_off(m, kc)) = hv;
+        *reinterpret_cast<uint4*>(lo + rec::k_off(m, kc)) = lv;
+    }
+}
+
+// =============================================================== intra-chunk kernel
+
+struct alignas(1024) PrepSmem {
+    // per dk half (12 KB): K_prev rows 0-31 | K rows 32-63 | Q rows 64-95, 128-byte rows,
+    // 128-byte swizzle.  Gram A = [K;Q] (rows 32-95), B = [K_prev;K] (rows 0-63).
+    uint8_t kq[2][12288];
+    // fp32 32 x 32 blocks, rows padded to 36 floats (16-byte rows, conflict-free vectors)
+    float Am[C][36];
+    float Pm[C][36];
+    float R3[C][36];  // diag(w) K K_prev^T diag(D_prev)
+    union {
+        struct {
+            float KK[C][36];  // K K^T
+            float KR[C][36];  // K K_prev^T
+            float QK[C][36];  // Q K^T
+        } g;
+        float X[C][100];  // [Wt | Tb | M]
+    } u;
+    alignas(16) float beta[C];
+    alignas(16) float G[C];
+    alignas(16) float eG[C];
+    alignas(16) float rk[C];
+    alignas(16) float rq[C];
+    alignas(16) float w[C];
+    alignas(16) float Gp[C];
+    alignas(16) float rkp[C];
+    alignas(16) float Dp[C];
+    uint64_t bar_tma, bar_mma;
+    uint32_t tmem;
+};
+
+constexpr int PREP_THREADS = 128;
+
+__global__ void __launch_bounds__(PREP_THREADS)
+intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+                   const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+                   const int32_t* __restrict__ cu_seqlens, int T, int nseq, int Hk, int Hv,
+                   uint8_t* __restrict__ ws) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    PrepSmem& sm = *reinterpret_cast<PrepSmem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int h = blockIdx.x % Hv;
+    const long long f = blockIdx.x / Hv;
+    int s, c;
+    if (!rec::locate(cu_seqlens, T, nseq, f, s, c)) return;  // past the last chunk
+    long long t0, t1;
+    seq_range(cu_seqlens, s, T, t0, t1);
+    const long long c0 = t0 + (long long)c * C;
+    const int n = (int)min((long long)C, t1 - c0);
+    const int kh = h / (Hv / Hk);
+    uint8_t* rc = ws + ((size_t)f * Hv + h) * rec::BYTES;
+    if ((smem_u32(smem_raw) & 1023u) != 0) {  // swizzled tiles need 1 KB alignment
+        if (tid == 0) atomicExch(&g_tc_status, 2);
+        return;
+    }
+
+    if (tid == 0) {
+        mbar_init(&sm.bar_tma, 1);
+        mbar_init(&sm.bar_mma, 1);
+        mbar_init_fence();
+        mbar_arrive_expect_tx(&sm.bar_tma, (c > 0 ? 6u : 4u) * 4096u);
+        for (int hf = 0; hf < 2; ++hf) {
+            const int x = kh * DK + 64 * hf;
+            if (c > 0) tma_load_2d(sm.kq[hf], &tm_k, x, (int)(c0 - C), &sm.bar_tma);
+            tma_load_2d(sm.kq[hf] + 4096, &tm_k, x, (int)c0, &sm.bar_tma);
+            tma_load_2d(sm.kq[hf] + 8192, &tm_q, x, (int)c0, &sm.bar_tma);
+        }
+    }
+    if (c == 0) {  // no previous chunk: its rows read as zero
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int idx = tid + PREP_THREADS * e;  // 512 x 16 B = both halves' 4 KB
+            *reinterpret_cast<uint4*>(sm.kq[idx >> 8] + 16 * (idx & 255)) = make_uint4(0, 0, 0, 0);
+        }
+        fence_async_smem();
+    }
+    if (warp == 0) tmem_alloc(&sm.tmem, 64);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+
+    // ---- gates of this chunk and of the previous one (warp 3); the rest wait for TMA
+    if (warp == 3) {
+        const float eA = expf(A_log[h]), dtb = dt_bias[h];
+        float g = 0.f, bt = 0.f;  // padding rows: no decay, no write
+        if (lane < n) {
+            const size_t th = (size_t)(c0 + lane) * Hv + h;
+            gates_fast(__bfloat162float(a[th]), __bfloat162float(b[th]), eA, dtb, g, bt);
+        }
+        const float Gc = warp_inclusive_scan(g, lane);
+        sm.beta[lane] = bt;
+        sm.G[lane] = Gc;
+        sm.eG[lane] = __expf(Gc);
+        float gp = 0.f;
+        if (c > 0) {
+            const size_t th = (size_t)(c0 - C + lane) * Hv + h;
+            float bp;
+            gates_fast(__bfloat162float(a[th]), __bfloat162float(b[th]), eA, dtb, gp, bp);
+        }
+        sm.Gp[lane] = warp_inclusive_scan(gp, lane);
+    }
+    bool ok = __syncthreads_and(mbar_wait(&sm.bar_tma, 0)) != 0;
+    // ---- Gram [K;Q] [K_prev;K]^T  (M = 64, N = 64, K = 128)
+    if (warp == 0) {
+        if (ok && elect_one()) {
+            const uint32_t base = smem_u32(sm.kq[0]);
+            const uint32_t id = idesc_bf16(64, 64, 0, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t off = (ks >> 2) * 12288 + (ks & 3) * 32;
+                mma_bf16(tmem, sdesc(base + 4096 + off, 16, 1024, kSw128),
+                         sdesc(base + off, 16, 1024, kSw128), id, ks > 0);
+            }
+            mma_commit(&sm.bar_mma);
+        }
+        __syncwarp();
+    }
+    // ---- inverse norms of Q and K_prev rows on the CUDA cores (thread pair per row; the
+    //      swizzle only permutes 16-byte pieces inside a row, which a sum ignores)
+    if (ok) {
+        const int r = tid >> 1, hf = tid & 1;
+        float ss = sumsq64(sm.kq[hf] + (r < 32 ? 0 : 4096) + r * 128);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if (hf == 0) {
+            if (r < 32)
+                sm.rkp[r] = inv_norm_fast(ss);
+            else
+                sm.rq[r - 32] = inv_norm_fast(ss) * rsqrtf((float)DK);
+        }
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&sm.bar_mma, 0)) != 0;
+    tc_fence_after();
+    if (ok) {
+        // accumulator row r = 16 w + lane (lanes 0-15): rows 0-31 K, 32-63 Q; columns
+        // 0-31 against K_prev, 32-63 against K
+        float v[64];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+            tmem_ld16(tmem + lane_base(warp) + 16 * q4, *reinterpret_cast<float(*)[16]>(&v[16 * q4]));
+        tmem_ld_wait();
+        if (lane < 16) {
+            const int r = 16 * warp + lane;
+            float* d0 = r < 32 ? sm.u.g.KR[r] : nullptr;
+            float* d1 = r < 32 ? sm.u.g.KK[r] : sm.u.g.QK[r - 32];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (d0)
+                    *reinterpret_cast<float4*>(d0 + 4 * q) =
+                        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                *reinterpret_cast<float4*>(d1 + 4 * q) =
+                    make_float4(v[32 + 4 * q], v[33 + 4 * q], v[34 + 4 * q], v[35 + 4 * q]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (!ok) {
+        if (tid == 0) atomicExch(&g_tc_status, 1);
+        return;
+    }
+
+    // ---- per-row scalars; E, D, gamma into the record
+    float* vec = reinterpret_cast<float*>(rc + rec::OFF_VEC);
+    if (tid < C) {
+        const int i = tid;
+        const float rk = inv_norm_fast(sm.u.g.KK[i][i]);
+        sm.rk[i] = rk;
+        sm.w[i] = sm.beta[i] * sm.eG[i] * rk;
+        vec[rec::VEC_E + i] = sm.eG[i] * sm.rq[i];
+        vec[rec::VEC_D + i] = __expf(sm.G[C - 1] - sm.G[i]) * rk;
+        if (i == 0) vec[rec::VEC_GAMMA] = __expf(sm.G[C - 1]);
+    } else if (tid < 2 * C) {
+        const int j = tid - C;
+        sm.Dp[j] = c > 0 ? __expf(sm.Gp[C - 1] - sm.Gp[j]) * sm.rkp[j] : 0.f;
+    }
+    __syncthreads();
+
+    // ---- A (strictly lower), P (lower), R3 = diag(w) K K_prev^T diag(D_prev):
+    //      thread -> row i, columns 8 cg .. 8 cg + 7
+    {
+        const int i = tid >> 2, j0 = 8 * (tid & 3);
+        const float Gi = sm.G[i], fa = sm.beta[i] * sm.rk[i], fp = sm.rq[i], wi = sm.w[i];
+        float am[8], pm[8], r3[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int j = j0 + q;
+            const float dec = __expf(Gi - sm.G[j]) * sm.rk[j];  // used only where j <= i
+            am[q] = j < i ? fa * sm.u.g.KK[i][j] * dec : 0.f;
+            pm[q] = j <= i ? fp * sm.u.g.QK[i][j] * dec : 0.f;
+            r3[q] = wi * sm.u.g.KR[i][j] * sm.Dp[j];
+        }
+#pragma unroll
+        for (int q = 0; q < 8; q += 4) {
+            *reinterpret_cast<float4*>(&sm.Am[i][j0 + q]) = make_float4(am[q], am[q + 1], am[q + 2], am[q + 3]);
+            *reinterpret_cast<float4*>(&sm.Pm[i][j0 + q]) = make_float4(pm[q], pm[q + 1], pm[q + 2], pm[q + 3]);
+            *reinterpret_cast<float4*>(&sm.R3[i][j0 + q]) = make_float4(r3[q], r3[q + 1], r3[q + 2], r3[q + 3]);
+        }
+    }
+    __syncthreads();
+
+    if (tid < 3 * C) {
+        // ---- forward substitution (I + A) x = rhs, one right-hand side per thread:
+        //      columns 0-31 diag(w), 32-63 diag(beta), 64-95 R3
+        const int mat = tid >> 5, jj = tid & 31;
+        float x[C];
+#pragma unroll
+        for (int i = 0; i < C; ++i) x[i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+            float bi;
+            if (mat == 0)
+                bi = i == jj ? sm.w[i] : 0.f;
+            else if (mat == 1)
+                bi = i == jj ? sm.beta[i] : 0.f;
+            else
+                bi = sm.R3[i][jj];
+            float s0 = bi, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+            for (int m = 0; m < (i & ~3); m += 4) {
+                const float4 av = *reinterpret_cast<const float4*>(&sm.Am[i][m]);
+                s0 -= av.x * x[m];
+                s1 -= av.y * x[m + 1];
+                s2 -= av.z * x[m + 2];
+                s3 -= av.w * x[m + 3];
+            }
+#pragma unroll
+            for (int m = i & ~3; m < i; ++m) s0 -= sm.Am[i][m] * x[m];
+            x[i] = (s0 + s1) + (s2 + s3);
+        }
+#pragma unroll
+        for (int i = 0; i < C; ++i) sm.u.X[i][tid] = x[i];
+    } else {
+        // ---- P image (warp 3, one row per lane)
+        store_image_row(sm.Pm[lane], 1.f, rc + rec::OFF_P, rc + rec::OFF_P + IMG, lane);
+    }
+    __syncthreads();
+    // ---- Wt, -Tb, M images: thread -> one row of one matrix
+    if (tid < 3 * C) {
+        const int mat = tid >> 5, i = tid & 31;
+        const uint32_t off = mat == 0 ? rec::OFF_WT : (mat == 1 ? rec::OFF_NTB : rec::OFF_M);
+        store_image_row(&sm.u.X[i][32 * mat], mat == 1 ? -1.f : 1.f, rc + off, rc + off + IMG, i);
+    }
+}
+
+// =============================================================== state-passing kernel
+
+constexpr int NT = 48;                      // dv columns per CTA
+constexpr int NTILES = (DV + NT - 1) / NT;  // 3 (the last a third empty)
+constexpr int NSTG = 3;                     // ring depth of tiles and records
+constexpr int SP_THREADS = 576;             // 18 warps
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t T_ACC1 = 0;    // 2 x 96, M = 64: [K_{c+1}; Q_c] [S_hi | S_lo]
+constexpr uint32_t T_ACC2 = 192;  // 2 x 96, M = 64: rows 0-31 -Delta_{c+1}, 32-63 P_c Delta_c
+constexpr uint32_t T_ACC3 = 384;  // 96, M = 128: K_c^T [DDelta_hi | DDelta_lo]
+constexpr uint32_t OPB = NT * C * 2;  // one K = 32 x N = 48 bf16 operand part (3072 B)
+
+// Warp roles
+//   0-7    S group: the state update S <- gamma S + K^T D Delta (row 32 (w % 4) + lane,
+//          24 columns per warp half) and the state's hi/lo operand
+//   8, 9, 12, 13   Y and Delta epilogues (accumulator rows 0-31)
+//   10, 11, 14, 15 output epilogue (accumulator rows 32-63)
+//   16     tensor-core issue (one lane)
+//   17     loads: TMA tiles and record images (one lane)
+struct alignas(1024) SpSmem {
+    // pair buffer b: per dk half (8 KB) rows 0-31 K_{b+1}, rows 32-63 Q_b; 128-byte swizzle
+    uint8_t kq[NSTG][16384];
+    uint8_t vt[NSTG][4096];  // V_c: 32 rows x 64 columns (48 used), 128-byte swizzle
+    struct Slot {            // operands of step c, K-major no swizzle, M = 64, K = 32
+        uint8_t wt[2][4096];   // [Wt_{c+1}; 0] hi, lo
+        uint8_t ntb[2][4096];  // [-Tb_{c+1}; 0] hi, lo
+        uint8_t mp[2][4096];   // [M_{c+1}; P_c] hi, lo
+    } slot[NSTG];
+    // thread-written MN-major no-swizzle B operands, hi part then lo part along N
+    uint8_t s_op[2 * NT * DK * 2];  // S: K = 128
+    uint8_t y_op[2 * OPB];          // Y
+    uint8_t d_op[2][2 * OPB];       // Delta (two buffers)
+    uint8_t dd_op[2][2 * OPB];      // diag(D) Delta
+    uint64_t kq_full[NSTG], kq_empty[NSTG];
+    uint64_t v_full[NSTG], v_empty[NSTG];
+    uint64_t slot_full[NSTG], slot_empty[NSTG];
+    uint64_t acc1_full[2], acc2_full[2], acc3_full;
+    uint64_t acc1_free[2], acc2_free[2];
+    uint64_t s_ready, y_ready, d_ready, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Waits as one warp: lane 0 polls (bounded), the verdict is broadcast; false once the
+// kernel is aborting.
+__device__ __forceinline__ bool warp_wait(int* abort, uint64_t* bar, uint32_t parity) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0 && *(volatile int*)abort == 0) {
+        if (mbar_wait(bar, parity))
+            ok = 1;
+        else
+            atomicExch(abort, 1);
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// Offset of K-row k, 8-column group g in an MN-major no-swizzle operand with `krows` rows.
+__device__ __forceinline__ uint32_t mn_off(int k, int g, int krows) {
+    return (uint32_t)(g * (krows / 8) * 128 + k * 16);
+}
+
+// 24 fp32 values (column groups g0 .. g0 + 2) of K-row k as the hi and lo parts of an
+// MN-major operand whose lo part starts `lo_off` bytes after the hi part.
+__device__ __forceinline__ void put24(uint8_t* op, uint32_t lo_off, int k, int g0, int krows,
+                                      const float (&v)[24]) {
+#pragma unroll
+    for (int g = 0; g < 3; ++g) {
+        uint4 hv, lv;
+        split2(v[8 * g + 0], v[8 * g + 1], hv.x, lv.x);
+        split2(v[8 * g + 2], v[8 * g + 3], hv.y, lv.y);
+        split2(v[8 * g + 4], v[8 * g + 5], hv.z, lv.z);
+        split2(v[8 * g + 6], v[8 * g + 7], hv.w, lv.w);
+        const uint32_t o = mn_off(k, g0 + g, krows);
+        *reinterpret_cast<uint4*>(op + o) = hv;
+        *reinterpret_cast<uint4*>(op + lo_off + o) = lv;
+    }
+}
+
+// hi + lo halves of a [hi | lo] accumulator (48 columns apart): 24 columns from taddr.
+__device__ __forceinline__ void ld_sum24(uint32_t taddr, float (&v)[24]) {
+    float h[24], l[24];
+    tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&h[0]));
+    tmem_ld8(taddr + 16, &h[16]);
+    tmem_ld16(taddr + NT, *reinterpret_cast<float(*)[16]>(&l[0]));
+    tmem_ld8(taddr + NT + 16, &l[16]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 24; ++i) v[i] = h[i] + l[i];
+}
+
+struct SpCtx {
+    int s, h, kh, Hv, col0, ncols, n;
+    long long t0, t1, rbase;  // token range, first record index of the sequence
+    const uint8_t* ws;
+    uint32_t tmem;
+    __device__ const float* vec(int c) const {
+        return reinterpret_cast<const float*>(ws + ((size_t)(rbase + c) * Hv + h) * rec::BYTES +
+                                              rec::OFF_VEC);
+    }
+    __device__ const uint8_t* record(int c) const {
+        return ws + ((size_t)(rbase + c) * Hv + h) * rec::BYTES;
+    }
+};
+
+// ------------------------------------------------------------------- loads (warp 17)
+__device__ void load_role(SpSmem& sm, const SpCtx& x, int lane, const CUtensorMap* tm_q,
+                          const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
+    int armed_kq[NSTG], armed_v[NSTG], armed_sl[NSTG];  // last use armed per ring entry
+    for (int r = 0; r < NSTG; ++r) armed_kq[r] = armed_v[r] = armed_sl[r] = -1;
+    for (int b = -1; b < x.n; ++b) {
+        const int r = (b + 1) % NSTG;
+        const int use = (b + 1) / NSTG;
+        // pair b: K_{b+1} and Q_b
+        if (use > 0 && !warp_wait(&sm.abort, &sm.kq_empty[r], (uint32_t)(use - 1) & 1u)) break;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&sm.kq_full[r], (b >= 0 ? 4u : 2u) * 4096u);
+            for (int hf = 0; hf < 2; ++hf) {
+                const int xx = x.kh * DK + 64 * hf;
+                tma_load_2d(sm.kq[r] + 8192 * hf, tm_k, xx, (int)(x.t0 + (long long)(b + 1) * C),
+                            &sm.kq_full[r]);
+                if (b >= 0)
+                    tma_load_2d(sm.kq[r] + 8192 * hf + 4096, tm_q, xx,
+                                (int)(x.t0 + (long long)b * C), &sm.kq_full[r]);
+            }
+        }
+        armed_kq[r] = use;
+        if (b + 1 < x.n) {
+            if (use > 0 && !warp_wait(&sm.abort, &sm.v_empty[r], (uint32_t)(use - 1) & 1u)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.v_full[r], 4096u);
+                tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, (int)(x.t0 + (long long)(b + 1) * C),
+                            &sm.v_full[r]);
+            }
+            armed_v[r] = use;
+        }
+        // record operands of step b
+        if (use > 0 && !warp_wait(&sm.abort, &sm.slot_empty[r], (uint32_t)(use - 1) & 1u)) break;
+        if (lane == 0) {
+            SpSmem::Slot& sl = sm.slot[r];
+            const uint32_t bytes = (b + 1 < x.n ? 6u * IMG : 0u) + (b >= 0 ? 2u * IMG : 0u);
+            mbar_arrive_expect_tx(&sm.slot_full[r], bytes);
+            if (b + 1 < x.n) {
+                const uint8_t* nx = x.record(b + 1);
+                bulk_load(sl.wt[0], nx + rec::OFF_WT, IMG, &sm.slot_full[r]);
+                bulk_load(sl.wt[1], nx + rec::OFF_WT + IMG, IMG, &sm.slot_full[r]);
+                bulk_load(sl.ntb[0], nx + rec::OFF_NTB, IMG, &sm.slot_full[r]);
+                bulk_load(sl.ntb[1], nx + rec::OFF_NTB + IMG, IMG, &sm.slot_full[r]);
+                bulk_load(sl.mp[0], nx + rec::OFF_M, IMG, &sm.slot_full[r]);
+                bulk_load(sl.mp[1], nx + rec::OFF_M + IMG, IMG, &sm.slot_full[r]);
+            }
+            if (b >= 0) {
+                const uint8_t* cu = x.record(b);
+                bulk_load(sl.mp[0] + IMG, cu + rec::OFF_P, IMG, &sm.slot_full[r]);
+                bulk_load(sl.mp[1] + IMG, cu + rec::OFF_P + IMG, IMG, &sm.slot_full[r]);
+            }
+        }
+        armed_sl[r] = use;
+        __syncwarp();
+    }
+    // every copy this warp started has landed before the CTA may exit
+    for (int r = 0; r < NSTG; ++r) {
+        if (lane == 0) {
+            if (armed_kq[r] >= 0) mbar_wait(&sm.kq_full[r], (uint32_t)armed_kq[r] & 1u);
+            if (armed_v[r] >= 0) mbar_wait(&sm.v_full[r], (uint32_t)armed_v[r] & 1u);
+            if (armed_sl[r] >= 0) mbar_wait(&sm.slot_full[r], (uint32_t)armed_sl[r] & 1u);
+        }
+    }
+    __syncwarp();
+}
+
+// ----------------------------------------------------------- tensor-core issue (warp 16)
+__device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
+    const uint32_t id96 = idesc_bf16(64, 2 * NT, 0, 1);
+    const uint32_t id48 = idesc_bf16(64, NT, 0, 1);
+    const uint32_t id_g3 = idesc_bf16(128, 2 * NT, 1, 1);
+    const uint64_t d_kq = sdesc(smem_u32(sm.kq[0]), 16, 1024, kSw128);    // [K;Q] K-major
+    const uint64_t d_kt = sdesc(smem_u32(sm.kq[0]), 8192, 1024, kSw128);  // K^T MN-major
+    const uint64_t d_vt = sdesc(smem_u32(sm.vt[0]), 8192, 1024, kSw128);  // V MN-major
+    const uint64_t d_s = sdesc(smem_u32(sm.s_op), 128, 2048, kSwNone);
+    const uint64_t d_y = sdesc(smem_u32(sm.y_op), 128, 512, kSwNone);
+    const uint64_t d_d = sdesc(smem_u32(sm.d_op[0]), 128, 512, kSwNone);
+    const uint64_t d_dd = sdesc(smem_u32(sm.dd_op[0]), 128, 512, kSwNone);
+    const uint64_t d_wt = sdesc(smem_u32(sm.slot[0].wt[0]), 128, 512, kSwNone);
+    const uint64_t d_ntb = sdesc(smem_u32(sm.slot[0].ntb[0]), 128, 512, kSwNone);
+    const uint64_t d_mp = sdesc(smem_u32(sm.slot[0].mp[0]), 128, 512, kSwNone);
+    constexpr uint32_t SLOT = sizeof(SpSmem::Slot);
+    constexpr uint32_t DBUF = 2 * OPB;
+    const bool leader = lane == 0;
+    int* ab = &sm.abort;
+    STAMP_INIT;
+
+    // G1a(b): acc1[(b+1)&1] = [K_{b+1}; Q_b] [S_b hi | lo]
+    auto g1a = [&](int b) {
+        const int r = (b + 1) % NSTG, x1 = (b + 1) & 1;
+        if (leader) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(x.tmem + T_ACC1 + 96 * x1,
+                         dadd(d_kq, r * 16384 + (ks >> 2) * 8192 + (ks & 3) * 32),
+                         dadd(d_s, ks * 256), id96, ks > 0);
+            mma_commit(&sm.acc1_full[x1]);
+        }
+        __syncwarp();
+    };
+
+    if (!warp_wait(ab, &sm.s_ready, 0)) goto drain;  // S_0 in place
+    if (!warp_wait(ab, &sm.kq_full[0], 0)) goto drain;
+    g1a(-1);
+    for (int b = -1; b < x.n; ++b) {
+        const int r = (b + 1) % NSTG, use = (b + 1) / NSTG;
+        const int x2 = (b + 1) & 1;
+        const uint32_t t2 = x.tmem + T_ACC2 + 96 * x2;
+        const bool nd = b + 1 < x.n;  // Delta_{b+1} needed
+        STAMP(b, 0);
+        if (b >= 1 && !warp_wait(ab, &sm.acc2_free[x2], (uint32_t)((b + 1) / 2 - 1) & 1u)) break;
+        STAMP(b, 1);
+        if (!warp_wait(ab, &sm.slot_full[r], (uint32_t)use & 1u)) break;
+        STAMP(b, 2);
+        bool first = true;
+        if (nd) {
+            if (!warp_wait(ab, &sm.v_full[r], (uint32_t)use & 1u)) break;
+            STAMP(b, 16);
+            tc_fence_after();
+            // U: [-Tb_{b+1}; 0] (hi -> columns 0-47, lo -> 48-95) V_{b+1}
+            if (leader) {
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                        mma_bf16(t2 + NT * part, dadd(d_ntb, r * SLOT + part * 4096 + ks * 256),
+                                 dadd(d_vt, r * 4096 + ks * 2048), id48, ks > 0);
+                mma_commit(&sm.v_empty[r]);
+                STAMP(b, 17);
+            }
+            __syncwarp();
+            first = false;
+        }
+        if (b >= 0) {
+            STAMP(b, 3);
+            if (!warp_wait(ab, &sm.d_ready, (uint32_t)b & 1u)) break;  // Delta_b, D Delta_b
+            STAMP(b, 4);
+            tc_fence_after();
+            if (leader) {
+                const uint64_t bd = dadd(d_d, (b & 1) * DBUF);
+                // [M_{b+1}; P_b] Delta_b
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(t2, dadd(d_mp, r * SLOT + ks * 256), dadd(bd, ks * 256), id96,
+                             first ? (ks > 0) : 1);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(t2, dadd(d_mp, r * SLOT + 4096 + ks * 256), dadd(bd, ks * 256), id48, 1);
+                // acc3 = K_b^T [D Delta_b hi | lo]   (K_b sits in pair buffer b - 1)
+                const uint64_t bdd = dadd(d_dd, (b & 1) * DBUF);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(x.tmem + T_ACC3, dadd(d_kt, (b % NSTG) * 16384 + ks * 2048),
+                             dadd(bdd, ks * 256), id_g3, ks > 0);
+                mma_commit(&sm.acc3_full);
+                mma_commit(&sm.kq_empty[b % NSTG]);
+                STAMP(b, 18);
+            }
+            __syncwarp();
+        }
+        if (nd) {
+            STAMP(b, 5);
+            if (!warp_wait(ab, &sm.y_ready, (uint32_t)(b + 1) & 1u)) break;  // Y_{b+1}
+            STAMP(b, 6);
+            tc_fence_after();
+            if (leader) {
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(t2, dadd(d_wt, r * SLOT + ks * 256), dadd(d_y, ks * 256), id96, 1);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(t2, dadd(d_wt, r * SLOT + 4096 + ks * 256), dadd(d_y, ks * 256), id48, 1);
+            }
+            __syncwarp();
+        }
+        if (leader) {
+            STAMP(b, 20);
+            mma_commit(&sm.acc2_full[x2]);
+            mma_commit(&sm.slot_empty[r]);
+            STAMP(b, 21);
+        }
+        __syncwarp();
+        if (nd) {
+            // G1a(b+1) needs S_{b+1} (phase b + 1 of s_ready) and a free acc1 buffer
+            STAMP(b, 7);
+            if (b >= 0 && !warp_wait(ab, &sm.s_ready, (uint32_t)(b + 1) & 1u)) break;
+            STAMP(b, 8);
+            const int x1 = (b + 2) & 1;
+            if (b + 2 >= 2 && !warp_wait(ab, &sm.acc1_free[x1], (uint32_t)((b + 2) / 2 - 1) & 1u)) break;
+            STAMP(b, 19);
+            if (!warp_wait(ab, &sm.kq_full[(b + 2) % NSTG], (uint32_t)((b + 2) / NSTG) & 1u)) break;
+            STAMP(b, 9);
+            tc_fence_after();
+            g1a(b + 1);
+        }
+    }
+drain:
+    // everything issued has completed before the CTA may exit
+    if (leader) {
+        mma_commit(&sm.drain);
+        mbar_wait(&sm.drain, 0);
+    }
+    __syncwarp();
+}
+
+// ------------------------------------------------------------ S group (warps 0-7)
+__device__ void s_role(SpSmem& sm, const SpCtx& x, int warp, int lane, const float* init_state,
+                       float* final_state) {
+    const int q = warp & 3, ch = warp >> 2;
+    const int k = 32 * q + lane;  // dk row
+    const int j0 = 24 * ch;       // first of this thread's 24 columns
+    STAMP_INIT;
+    const uint32_t tl = x.tmem + lane_base(warp);
+    constexpr uint32_t LO = NT * DK * 2;
+    const size_t srow = (((size_t)x.s * x.Hv + x.h) * DK + k) * DV + x.col0 + j0;
+    const int nvalid = DV - (x.col0 + j0);  // columns past dv are computed, never stored
+    float Sm[24];
+#pragma unroll
+    for (int j = 0; j < 24; j += 4) {
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (init_state && j < nvalid) t = *reinterpret_cast<const float4*>(init_state + srow + j);
+        Sm[j] = t.x; Sm[j + 1] = t.y; Sm[j + 2] = t.z; Sm[j + 3] = t.w;
+    }
+    put24(sm.s_op, LO, k, 3 * ch, DK, Sm);
+    fence_async_smem();
+    mbar_arrive(&sm.s_ready);
+    bool ok = true;
+    // the per-chunk scalars come from the workspace; each is loaded a step before its use
+    float gam_next = x.vec(0)[rec::VEC_GAMMA];
+    for (int b = 0; b < x.n; ++b) {
+        const float gam = gam_next;
+        if (b + 1 < x.n) gam_next = x.vec(b + 1)[rec::VEC_GAMMA];
+        if (!warp_wait(&sm.abort, &sm.acc3_full, (uint32_t)b & 1u)) { ok = false; break; }
+        if (warp == 0) STAMP(b, 10);
+        tc_fence_after();
+        float v[24];
+        ld_sum24(tl + T_ACC3 + j0, v);
+#pragma unroll
+        for (int j = 0; j < 24; ++j) Sm[j] = gam * Sm[j] + v[j];
+        if (b + 1 < x.n) {
+            put24(sm.s_op, LO, k, 3 * ch, DK, Sm);
+            fence_async_smem();
+        }
+        tc_fence_before();
+        if (warp == 0) STAMP(b, 11);
+        mbar_arrive(&sm.s_ready);
+    }
+    if (ok && final_state && *(volatile int*)&sm.abort == 0) {
+#pragma unroll
+        for (int j = 0; j < 24; j += 4)
+            if (j < nvalid)
+                *reinterpret_cast<float4*>(final_state + srow + j) =
+                    make_float4(Sm[j], Sm[j + 1], Sm[j + 2], Sm[j + 3]);
+    }
+}
+
+// -------------------------------------------- Y and Delta epilogues (warps 8, 9, 12, 13)
+__device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
+    const int q = warp & 3, ch = (warp - 8) >> 2;
+    const int r = 16 * q + lane;  // accumulator row (valid for lane < 16)
+    const int j0 = 24 * ch;
+    const uint32_t tl = x.tmem + lane_base(warp);
+    STAMP_INIT;
+    // per-chunk scalars, loaded a step before their use
+    float gam_next = 1.f, d_next = lane < 16 ? x.vec(0)[rec::VEC_D + r] : 0.f;
+    for (int b = -1; b + 1 < x.n; ++b) {
+        const int x1 = (b + 1) & 1;
+        // Y_{b+1} = gamma_b K_{b+1} S_b
+        const float gam = gam_next, d = d_next;
+        if (b + 2 < x.n) {
+            gam_next = x.vec(b + 1)[rec::VEC_GAMMA];
+            d_next = lane < 16 ? x.vec(b + 2)[rec::VEC_D + r] : 0.f;
+        }
+        if (!warp_wait(&sm.abort, &sm.acc1_full[x1], (uint32_t)((b + 1) >> 1) & 1u)) return;
+        if (warp == 8) STAMP(b + 1, 12);
+        tc_fence_after();
+        float v[24];
+        ld_sum24(tl + T_ACC1 + 96 * x1 + j0, v);
+#pragma unroll
+        for (int j = 0; j < 24; ++j) v[j] *= gam;
+        if (lane < 16) put24(sm.y_op, OPB, r, 3 * ch, C, v);
+        fence_async_smem();
+        tc_fence_before();
+        if (warp == 8) STAMP(b + 1, 13);
+        mbar_arrive(&sm.y_ready);
+        mbar_arrive(&sm.acc1_free[x1]);
+        // Delta_{b+1} = -acc2 rows 0-31; D Delta_{b+1}
+        if (!warp_wait(&sm.abort, &sm.acc2_full[x1], (uint32_t)((b + 1) >> 1) & 1u)) return;
+        if (warp == 8) STAMP(b + 1, 14);
+        tc_fence_after();
+        ld_sum24(tl + T_ACC2 + 96 * x1 + j0, v);
+        float w[24];
+#pragma unroll
+        for (int j = 0; j < 24; ++j) {
+            v[j] = -v[j];
+            w[j] = d * v[j];
+        }
+        const int nb = (b + 1) & 1;
+        if (lane < 16) {
+            put24(sm.d_op[nb], OPB, r, 3 * ch, C, v);
+            put24(sm.dd_op[nb], OPB, r, 3 * ch, C, w);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (warp == 8) STAMP(b + 1, 15);
+        mbar_arrive(&sm.d_ready);
+        mbar_arrive(&sm.acc2_free[x1]);
+    }
+}
+
+// ---------------------------------------------- output epilogue (warps 10, 11, 14, 15)
+__device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __restrict__ out) {
+    const int q = warp & 3, ch = (warp - 8) >> 2;
+    const int i = 16 * (q - 2) + lane;  // chunk position (valid for lane < 16)
+    const int j0 = 24 * ch;
+    STAMP_INIT;
+    const uint32_t tl = x.tmem + lane_base(warp);
+    const int nvalid = DV - (x.col0 + j0);
+    // step -1 produces no output; its accumulators are released at once
+    mbar_arrive(&sm.acc1_free[0]);
+    mbar_arrive(&sm.acc2_free[0]);
+    float e_next = lane < 16 ? x.vec(0)[rec::VEC_E + i] : 0.f;  // loaded a step ahead
+    for (int b = 0; b < x.n; ++b) {
+        const int x1 = (b + 1) & 1;
+        const uint32_t ph = (uint32_t)((b + 1) >> 1) & 1u;
+        const float e = e_next;
+        if (b + 1 < x.n) e_next = lane < 16 ? x.vec(b + 1)[rec::VEC_E + i] : 0.f;
+        if (!warp_wait(&sm.abort, &sm.acc1_full[x1], ph)) return;
+        tc_fence_after();
+        float qs[24];
+        ld_sum24(tl + T_ACC1 + 96 * x1 + j0, qs);
+        tc_fence_before();
+        mbar_arrive(&sm.acc1_free[x1]);
+        if (!warp_wait(&sm.abort, &sm.acc2_full[x1], ph)) return;
+        tc_fence_after();
+        float pd[24];
+        ld_sum24(tl + T_ACC2 + 96 * x1 + j0, pd);
+        tc_fence_before();
+        mbar_arrive(&sm.acc2_free[x1]);
+        const long long c0 = x.t0 + (long long)b * C;
+        if (lane < 16 && c0 + i < x.t1) {
+            float* op = out + ((size_t)(c0 + i) * x.Hv + x.h) * DV + x.col0 + j0;
+#pragma unroll
+            for (int j = 0; j < 24; j += 4)
+                if (j < nvalid)
+                    *reinterpret_cast<float4*>(op + j) =
+                    make_float4(e * qs[j] + pd[j], e * qs[j + 1] + pd[j + 1],
+                                e * qs[j + 2] + pd[j + 2], e * qs[j + 3] + pd[j + 3]);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(SP_THREADS, 1)
+state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const uint8_t* __restrict__ ws,
+                  const float* init_state, float* __restrict__ out, float* final_state,
+                  const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    SpSmem& sm = *reinterpret_cast<SpSmem*>(smem_raw);
+    const int tile = blockIdx.x % NTILES;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    SpCtx x;
+    x.h = (blockIdx.x / NTILES) % Hv;
+    x.s = blockIdx.x / (NTILES * Hv);
+    x.kh = x.h / (Hv / Hk);
+    x.Hv = Hv;
+    x.col0 = tile * NT;
+    x.ncols = min(NT, DV - x.col0);
+    seq_range(cu_seqlens, x.s, T, x.t0, x.t1);
+    x.n = (int)((x.t1 - x.t0 + C - 1) / C);
+    x.rbase = rec::chunk_base(cu_seqlens, x.s, T);
+    x.ws = ws;
+
+    if (x.n == 0) {  // empty sequence: the final state is the initial one
+        if (final_state && tid < DK) {
+            const size_t row = (((size_t)x.s * Hv + x.h) * DK + tid) * DV + x.col0;
+            for (int j = 0; j < x.ncols; j += 4)
+                *reinterpret_cast<float4*>(final_state + row + j) =
+                    init_state ? *reinterpret_cast<const float4*>(init_state + row + j)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        return;
+    }
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (tid == 0) atomicExch(&g_tc_status, 2);
+        return;
+    }
+    if (tid == 0) {
+        for (int i = 0; i < NSTG; ++i) {
+            mbar_init(&sm.kq_full[i], 1);
+            mbar_init(&sm.kq_empty[i], 1);
+            mbar_init(&sm.v_full[i], 1);
+            mbar_init(&sm.v_empty[i], 1);
+            mbar_init(&sm.slot_full[i], 1);
+            mbar_init(&sm.slot_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.acc1_full[i], 1);
+            mbar_init(&sm.acc2_full[i], 1);
+            mbar_init(&sm.acc1_free[i], 256);
+            mbar_init(&sm.acc2_free[i], 256);
+        }
+        mbar_init(&sm.acc3_full, 1);
+        mbar_init(&sm.s_ready, 256);
+        mbar_init(&sm.y_ready, 128);
+        mbar_init(&sm.d_ready, 128);
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        mbar_init_fence();
+        tma_prefetch_map(&tm_q);
+        tma_prefetch_map(&tm_k);
+        tma_prefetch_map(&tm_v);
+    }
+    // rows 32-63 of the [Wt; 0] and [-Tb; 0] operands stay zero
+    for (int e = tid; e < NSTG * 4 * (IMG / 16); e += SP_THREADS) {
+        const int sl = e / (4 * (IMG / 16)), rem = e % (4 * (IMG / 16));
+        const int which = rem / (IMG / 16), off = 16 * (rem % (IMG / 16));
+        uint8_t* base = which < 2 ? sm.slot[sl].wt[which] : sm.slot[sl].ntb[which - 2];
+        *reinterpret_cast<uint4*>(base + IMG + off) = make_uint4(0, 0, 0, 0);
+    }
+    fence_async_smem();
+    if (warp == 0) tmem_alloc(&sm.tmem_base, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    x.tmem = sm.tmem_base;
+
+    if (warp < 8)
+        s_role(sm, x, warp, lane, init_state, final_state);
+    else if (warp < 16)
+        ((warp & 3) < 2) ? d_role(sm, x, warp, lane) : o_role(sm, x, warp, lane, out);
+    else if (warp == 16)
+        mma_role(sm, x, lane);
+    else
+        load_role(sm, x, lane, &tm_q, &tm_k, &tm_v);
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(x.tmem, TMEM_COLS);
+    if (tid == 0 && sm.abort) atomicExch(&g_tc_status, 1);
+}
+
+// ---------------------------------------------------------------- workspace
+
+// A private stream-ordered pool per device; memory returned to it stays cached until
+// gdr_release_workspace() trims it.
+struct PoolSet {
+    std::mutex mu;
+    cudaMemPool_t pool[64] = {};
+    bool made[64] = {};
+};
+PoolSet& pools() {
+    static PoolSet p;
+    return p;
+}
+
+}  // namespace
+
+cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    PoolSet& ps = pools();
+    std::lock_guard<std::mutex> lock(ps.mu);
+    if (!ps.made[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        e = cudaMemPoolCreate(&ps.pool[dev], &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = ~0ull;  // keep freed memory for the next call
+        cudaMemPoolSetAttribute(ps.pool[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+        ps.made[dev] = true;
+    }
+    return cudaMallocFromPoolAsync(ptr, bytes, ps.pool[dev], stream);
+}
+
+void workspace_release() {
+    PoolSet& ps = pools();
+    std::lock_guard<std::mutex> lock(ps.mu);
+    for (int d = 0; d < 64; ++d)
+        if (ps.made[d]) cudaMemPoolTrimTo(ps.pool[d], 0);
+}
+
+size_t prefill_tc_workspace_bytes(const FwdParams& p) {
+    return (size_t)rec::max_records(p.cu_seqlens != nullptr, p.nseq, p.T) * p.Hv * rec::BYTES;
+}
+
+cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stream) {
+    if (p.in != InType::BF16 || p.dk != DK || p.dv != DV || p.chunk != C)
+        return cudaErrorNotSupported;
+    const long long tokens = p.cu_seqlens ? (long long)p.T : (long long)p.nseq * p.T;
+    if (tokens <= 0 || tokens >= (1LL << 31) - 64) return cudaErrorNotSupported;
+    CUtensorMap mq, mk, mv;
+    if (!make_bf16_map(&mq, p.q, (uint64_t)p.Hk * DK, tokens) ||
+        !make_bf16_map(&mk, p.k, (uint64_t)p.Hk * DK, tokens) ||
+        !make_bf16_map(&mv, p.v, (uint64_t)p.Hv * DV, tokens))
+        return cudaErrorInvalidValue;
+    const long long nrec = rec::max_records(p.cu_seqlens != nullptr, p.nseq, p.T);
+    cudaError_t e = cudaFuncSetAttribute(intra_chunk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(PrepSmem));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(SpSmem));
+    if (e != cudaSuccess) return e;
+    intra_chunk_kernel<<<(unsigned)(nrec * p.Hv), PREP_THREADS, sizeof(PrepSmem), stream>>>(
+        mq, mk, (const __nv_bfloat16*)p.a, (const __nv_bfloat16*)p.b, p.A_log, p.dt_bias,
+        p.cu_seqlens, p.T, p.nseq, p.Hk, p.Hv, (uint8_t*)ws);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    state_pass_kernel<<<(unsigned)(p.nseq * p.Hv * NTILES), SP_THREADS, sizeof(SpSmem), stream>>>(
+        mq, mk, mv, (const uint8_t*)ws, p.init_state, p.out, p.final_state, p.cu_seqlens, p.T,
+        p.Hk, p.Hv);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_tc(const FwdParams& p, cudaStream_t stream) {
+    if (p.in != InType::BF16 || p.dk != DK || p.dv != DV || p.chunk != C)
+        return cudaErrorNotSupported;
+    void* ws = nullptr;
+    cudaError_t e = workspace_alloc(&ws, prefill_tc_workspace_bytes(p), stream);
+    if (e != cudaSuccess) return e;
+    e = launch_prefill_tc_ws(p, ws, stream);
+    const cudaError_t f = cudaFreeAsync(ws, stream);
+    return e != cudaSuccess ? e : f;
+}
+
+#ifdef GDR_TC_STAMP
+void set_stamp_buffer(long long* p) { cudaMemcpyToSymbol(g_stamp, &p, sizeof(p)); }
+#endif
+
+int read_and_clear_tc_status() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_status, sizeof(int)) != cudaSuccess) return -1;
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_tc_status, &zero, sizeof(int));
+    }
+    return v;
+}
+
+}  // namespace gdr

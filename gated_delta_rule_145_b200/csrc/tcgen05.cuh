@@ -30,6 +30,10 @@ namespace gdr {
 namespace tc {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+#ifndef GDR_POLL_SLEEP_NS
+#define GDR_POLL_SLEEP_NS 20
+#endif
+constexpr uint32_t kPollSleepNs = GDR_POLL_SLEEP_NS;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -105,12 +109,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity; false if it did not complete in time.
+// Out of line: one copy of the polling loop serves every call site, which keeps the
+// kernels' code small (code that is not resident in the instruction cache costs far more
+// than the call).
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity);
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity);
+}
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer();
+    // kept rolled: every call site inlines this loop, and an unrolled copy per site
+    // would swell the kernels past the instruction cache
     for (;;) {
-        for (int i = 0; i < 64; ++i)
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i) {
             if (mbar_try_wait(bar, parity)) return true;
+            __nanosleep(kPollSleepNs);  // leave the issue slots to the working warps
+        }
         if (globaltimer() - t0 > kWaitLimitNs) return false;
     }
 }
@@ -124,6 +140,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Plain bulk copy global -> shared (this CTA): `bytes` (a multiple of 16) from a 16-byte
+// aligned global address, completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -172,6 +199,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
         : "r"(taddr));
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_ld_wait() {

@@ -35,7 +35,13 @@
  *     abort; they return one of the GDR_* codes below.  GDR_ERR_CUDA reports a launch
  *     error taken from cudaGetLastError (which clears it).
  *   - Supported head sizes: dk == dv in {32, 64, 128}; chunk == 32.
- *   - The library allocates no device memory: all intermediates stay on chip.
+ *   - Memory: the bf16 chunked prefill at dk = dv = 128 needs a workspace of
+ *     16896 bytes per (chunk, value head) -- 208 MB for T = 8192, Hv = 48 -- which the
+ *     library takes, per call, from a private stream-ordered pool of the current device
+ *     (cudaMallocFromPoolAsync on `stream`, returned with cudaFreeAsync on the same
+ *     stream once the call's kernels are enqueued).  Freed memory stays cached in the pool
+ *     for later calls until gdr_release_workspace().  Calls on different streams get
+ *     different workspace memory.  No other call allocates device memory.
  */
 #ifndef GDR_H_
 #define GDR_H_
@@ -59,6 +65,7 @@ typedef void* gdr_stream_t; /* cudaStream_t */
 #define GDR_ERR_SHAPE (-2)       /* B, T, Hk, Hv inconsistent (e.g. Hv % Hk != 0) */
 #define GDR_ERR_UNSUPPORTED (-3) /* head size or chunk size not built */
 #define GDR_ERR_ALIGN (-4)       /* a pointer is not aligned as stated above */
+#define GDR_ERR_OOM (-5)         /* the prefill workspace could not be allocated */
 #define GDR_ERR_CUDA (-6)        /* a kernel launch failed */
 #define GDR_ERR_TIMEOUT (-7)     /* a kernel gave up a bounded on-chip wait (see below) */
 
@@ -138,6 +145,14 @@ GDR_API int gdr_prefill_recurrent_f32(const float* q, const float* k, const floa
  * The timeout record is cleared by the call.
  */
 GDR_API int gdr_device_status(gdr_stream_t stream);
+
+/*
+ * Returns the workspace memory cached by earlier gdr_prefill_chunked calls to the system
+ * (every device's pool is trimmed to zero).  Memory still in use by enqueued work is
+ * released once that work completes.  No counterpart on the pages: it manages this
+ * library's own cache.
+ */
+GDR_API void gdr_release_workspace(void);
 
 /* A static, human-readable name for a GDR_* status code. */
 GDR_API const char* gdr_status_string(int status);
