@@ -49,19 +49,6 @@ namespace gdr {
 // Set when a bounded wait inside a kernel expired (read by gdr_device_status()).
 __device__ int g_tc_status = 0;
 
-#ifdef GDR_TC_STAMP
-// Cycle stamps of CTA 0 of the state-passing kernel, steps 0-63 (debug builds only).
-__device__ long long* g_stamp = nullptr;
-#define STAMP(b, k)                                                                       \
-    do {                                                                                  \
-        if (stamp_ptr && (b) >= 0 && (b) < 64 && (threadIdx.x & 31) == 0)                 \
-            stamp_ptr[(b) * 32 + (k)] = clock64();                                        \
-    } while (0)
-#define STAMP_INIT long long* stamp_ptr = blockIdx.x == 0 ? g_stamp : nullptr
-#else
-#define STAMP(b, k)
-#define STAMP_INIT
-#endif
 
 namespace {
 
@@ -413,29 +400,25 @@ struct alignas(1024) SpSmem {
     uint8_t y_op[2 * OPB];          // Y
     uint8_t d_op[2][2 * OPB];       // Delta (two buffers)
     uint8_t dd_op[2][2 * OPB];      // diag(D) Delta
-    uint64_t kq_full[NSTG], kq_empty[NSTG];
-    uint64_t v_full[NSTG], v_empty[NSTG];
-    uint64_t slot_full[NSTG], slot_empty[NSTG];
+    // step b's loads (pair b, V_{b+1}, record operands of step b) share ring entry
+    // (b + 1) % NSTG and one full / one empty barrier
+    uint64_t step_full[NSTG], step_empty[NSTG];
     uint64_t acc1_full[2], acc2_full[2], acc3_full;
-    uint64_t acc1_free[2], acc2_free[2];
+    // s_ready: S group wrote S_{b+1}.  y_ready: Y_{b+1} written and acc1 of step b read.
+    // d_ready: Delta_{b+1} written and acc2 of step b read.
     uint64_t s_ready, y_ready, d_ready, drain;
     uint32_t tmem_base;
     int abort;
 };
 
-// Waits as one warp: lane 0 polls (bounded), the verdict is broadcast; false once the
-// kernel is aborting.
+// Waits as one converged warp (every lane runs the same polls, so the lanes agree);
+// false once the kernel is aborting.  The fast path is a single non-blocking test.
 __device__ __forceinline__ bool warp_wait(int* abort, uint64_t* bar, uint32_t parity) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0 && *(volatile int*)abort == 0) {
-        if (mbar_wait(bar, parity))
-            ok = 1;
-        else
-            atomicExch(abort, 1);
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    __syncwarp();
-    return ok != 0;
+    if (mbar_test(bar, parity)) return true;
+    if (*(volatile int*)abort) return false;
+    if (mbar_wait_slow(bar, parity)) return true;
+    atomicExch(abort, 1);
+    return false;
 }
 
 // Offset of K-row k, 8-column group g in an MN-major no-swizzle operand with `krows` rows.
@@ -489,66 +472,50 @@ struct SpCtx {
 // ------------------------------------------------------------------- loads (warp 17)
 __device__ void load_role(SpSmem& sm, const SpCtx& x, int lane, const CUtensorMap* tm_q,
                           const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
-    int armed_kq[NSTG], armed_v[NSTG], armed_sl[NSTG];  // last use armed per ring entry
-    for (int r = 0; r < NSTG; ++r) armed_kq[r] = armed_v[r] = armed_sl[r] = -1;
+    int armed = -2;  // last step whose loads were issued
     for (int b = -1; b < x.n; ++b) {
         const int r = (b + 1) % NSTG;
         const int use = (b + 1) / NSTG;
-        // pair b: K_{b+1} and Q_b
-        if (use > 0 && !warp_wait(&sm.abort, &sm.kq_empty[r], (uint32_t)(use - 1) & 1u)) break;
+        // ring entry r last served step b - NSTG, released once G3(b - NSTG + 1) has read
+        // its K tile
+        if (use > 0 && !warp_wait(&sm.abort, &sm.step_empty[r], (uint32_t)(use - 1) & 1u)) break;
         if (lane == 0) {
-            mbar_arrive_expect_tx(&sm.kq_full[r], (b >= 0 ? 4u : 2u) * 4096u);
+            const bool next = b + 1 < x.n;
+            const uint32_t bytes = (b >= 0 ? 4u : 2u) * 4096u + (next ? 4096u + 6u * IMG : 0u) +
+                                   (b >= 0 ? 2u * IMG : 0u);
+            uint64_t* bar = &sm.step_full[r];
+            mbar_arrive_expect_tx(bar, bytes);
+            const int y1 = (int)(x.t0 + (long long)(b + 1) * C), y0 = y1 - C;
+            // pair b: K_{b+1} and Q_b
             for (int hf = 0; hf < 2; ++hf) {
                 const int xx = x.kh * DK + 64 * hf;
-                tma_load_2d(sm.kq[r] + 8192 * hf, tm_k, xx, (int)(x.t0 + (long long)(b + 1) * C),
-                            &sm.kq_full[r]);
-                if (b >= 0)
-                    tma_load_2d(sm.kq[r] + 8192 * hf + 4096, tm_q, xx,
-                                (int)(x.t0 + (long long)b * C), &sm.kq_full[r]);
+                tma_load_2d(sm.kq[r] + 8192 * hf, tm_k, xx, y1, bar);
+                if (b >= 0) tma_load_2d(sm.kq[r] + 8192 * hf + 4096, tm_q, xx, y0, bar);
             }
-        }
-        armed_kq[r] = use;
-        if (b + 1 < x.n) {
-            if (use > 0 && !warp_wait(&sm.abort, &sm.v_empty[r], (uint32_t)(use - 1) & 1u)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.v_full[r], 4096u);
-                tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, (int)(x.t0 + (long long)(b + 1) * C),
-                            &sm.v_full[r]);
-            }
-            armed_v[r] = use;
-        }
-        // record operands of step b
-        if (use > 0 && !warp_wait(&sm.abort, &sm.slot_empty[r], (uint32_t)(use - 1) & 1u)) break;
-        if (lane == 0) {
             SpSmem::Slot& sl = sm.slot[r];
-            const uint32_t bytes = (b + 1 < x.n ? 6u * IMG : 0u) + (b >= 0 ? 2u * IMG : 0u);
-            mbar_arrive_expect_tx(&sm.slot_full[r], bytes);
-            if (b + 1 < x.n) {
+            if (next) {
+                tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, y1, bar);
                 const uint8_t* nx = x.record(b + 1);
-                bulk_load(sl.wt[0], nx + rec::OFF_WT, IMG, &sm.slot_full[r]);
-                bulk_load(sl.wt[1], nx + rec::OFF_WT + IMG, IMG, &sm.slot_full[r]);
-                bulk_load(sl.ntb[0], nx + rec::OFF_NTB, IMG, &sm.slot_full[r]);
-                bulk_load(sl.ntb[1], nx + rec::OFF_NTB + IMG, IMG, &sm.slot_full[r]);
-                bulk_load(sl.mp[0], nx + rec::OFF_M, IMG, &sm.slot_full[r]);
-                bulk_load(sl.mp[1], nx + rec::OFF_M + IMG, IMG, &sm.slot_full[r]);
+                bulk_load(sl.wt[0], nx + rec::OFF_WT, IMG, bar);
+                bulk_load(sl.wt[1], nx + rec::OFF_WT + IMG, IMG, bar);
+                bulk_load(sl.ntb[0], nx + rec::OFF_NTB, IMG, bar);
+                bulk_load(sl.ntb[1], nx + rec::OFF_NTB + IMG, IMG, bar);
+                bulk_load(sl.mp[0], nx + rec::OFF_M, IMG, bar);
+                bulk_load(sl.mp[1], nx + rec::OFF_M + IMG, IMG, bar);
             }
             if (b >= 0) {
                 const uint8_t* cu = x.record(b);
-                bulk_load(sl.mp[0] + IMG, cu + rec::OFF_P, IMG, &sm.slot_full[r]);
-                bulk_load(sl.mp[1] + IMG, cu + rec::OFF_P + IMG, IMG, &sm.slot_full[r]);
+                bulk_load(sl.mp[0] + IMG, cu + rec::OFF_P, IMG, bar);
+                bulk_load(sl.mp[1] + IMG, cu + rec::OFF_P + IMG, IMG, bar);
             }
         }
-        armed_sl[r] = use;
         __syncwarp();
+        armed = b;
     }
-    // every copy this warp started has landed before the CTA may exit
-    for (int r = 0; r < NSTG; ++r) {
-        if (lane == 0) {
-            if (armed_kq[r] >= 0) mbar_wait(&sm.kq_full[r], (uint32_t)armed_kq[r] & 1u);
-            if (armed_v[r] >= 0) mbar_wait(&sm.v_full[r], (uint32_t)armed_v[r] & 1u);
-            if (armed_sl[r] >= 0) mbar_wait(&sm.slot_full[r], (uint32_t)armed_sl[r] & 1u);
-        }
-    }
+    // every copy this warp started has landed before the CTA may exit (entries older than
+    // the last NSTG steps were consumed before their reuse)
+    for (int b = max(-1, armed - NSTG + 1); b <= armed; ++b)
+        mbar_wait(&sm.step_full[(b + 1) % NSTG], (uint32_t)((b + 1) / NSTG) & 1u);
     __syncwarp();
 }
 
@@ -571,7 +538,6 @@ __device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
     constexpr uint32_t DBUF = 2 * OPB;
     const bool leader = lane == 0;
     int* ab = &sm.abort;
-    STAMP_INIT;
 
     // G1a(b): acc1[(b+1)&1] = [K_{b+1}; Q_b] [S_b hi | lo]
     auto g1a = [&](int b) {
@@ -588,23 +554,19 @@ __device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
     };
 
     if (!warp_wait(ab, &sm.s_ready, 0)) goto drain;  // S_0 in place
-    if (!warp_wait(ab, &sm.kq_full[0], 0)) goto drain;
+    if (!warp_wait(ab, &sm.step_full[0], 0)) goto drain;
     g1a(-1);
     for (int b = -1; b < x.n; ++b) {
         const int r = (b + 1) % NSTG, use = (b + 1) / NSTG;
         const int x2 = (b + 1) & 1;
         const uint32_t t2 = x.tmem + T_ACC2 + 96 * x2;
         const bool nd = b + 1 < x.n;  // Delta_{b+1} needed
-        STAMP(b, 0);
-        if (b >= 1 && !warp_wait(ab, &sm.acc2_free[x2], (uint32_t)((b + 1) / 2 - 1) & 1u)) break;
-        STAMP(b, 1);
-        if (!warp_wait(ab, &sm.slot_full[r], (uint32_t)use & 1u)) break;
-        STAMP(b, 2);
+        // acc2[x2] was last read in step b - 2, covered by d_ready phase b - 1 (waited in
+        // step b - 1)
+        if (!warp_wait(ab, &sm.step_full[r], (uint32_t)use & 1u)) break;
+        tc_fence_after();
         bool first = true;
         if (nd) {
-            if (!warp_wait(ab, &sm.v_full[r], (uint32_t)use & 1u)) break;
-            STAMP(b, 16);
-            tc_fence_after();
             // U: [-Tb_{b+1}; 0] (hi -> columns 0-47, lo -> 48-95) V_{b+1}
             if (leader) {
 #pragma unroll
@@ -613,16 +575,12 @@ __device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
                     for (int ks = 0; ks < 2; ++ks)
                         mma_bf16(t2 + NT * part, dadd(d_ntb, r * SLOT + part * 4096 + ks * 256),
                                  dadd(d_vt, r * 4096 + ks * 2048), id48, ks > 0);
-                mma_commit(&sm.v_empty[r]);
-                STAMP(b, 17);
             }
             __syncwarp();
             first = false;
         }
         if (b >= 0) {
-            STAMP(b, 3);
             if (!warp_wait(ab, &sm.d_ready, (uint32_t)b & 1u)) break;  // Delta_b, D Delta_b
-            STAMP(b, 4);
             tc_fence_after();
             if (leader) {
                 const uint64_t bd = dadd(d_d, (b & 1) * DBUF);
@@ -641,15 +599,12 @@ __device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
                     mma_bf16(x.tmem + T_ACC3, dadd(d_kt, (b % NSTG) * 16384 + ks * 2048),
                              dadd(bdd, ks * 256), id_g3, ks > 0);
                 mma_commit(&sm.acc3_full);
-                mma_commit(&sm.kq_empty[b % NSTG]);
-                STAMP(b, 18);
+                mma_commit(&sm.step_empty[b % NSTG]);  // step b - 1's loads all read
             }
             __syncwarp();
         }
         if (nd) {
-            STAMP(b, 5);
             if (!warp_wait(ab, &sm.y_ready, (uint32_t)(b + 1) & 1u)) break;  // Y_{b+1}
-            STAMP(b, 6);
             tc_fence_after();
             if (leader) {
 #pragma unroll
@@ -662,22 +617,14 @@ __device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
             __syncwarp();
         }
         if (leader) {
-            STAMP(b, 20);
             mma_commit(&sm.acc2_full[x2]);
-            mma_commit(&sm.slot_empty[r]);
-            STAMP(b, 21);
         }
         __syncwarp();
         if (nd) {
             // G1a(b+1) needs S_{b+1} (phase b + 1 of s_ready) and a free acc1 buffer
-            STAMP(b, 7);
             if (b >= 0 && !warp_wait(ab, &sm.s_ready, (uint32_t)(b + 1) & 1u)) break;
-            STAMP(b, 8);
-            const int x1 = (b + 2) & 1;
-            if (b + 2 >= 2 && !warp_wait(ab, &sm.acc1_free[x1], (uint32_t)((b + 2) / 2 - 1) & 1u)) break;
-            STAMP(b, 19);
-            if (!warp_wait(ab, &sm.kq_full[(b + 2) % NSTG], (uint32_t)((b + 2) / NSTG) & 1u)) break;
-            STAMP(b, 9);
+            // acc1 of step b - 1 was read before y_ready phase b (waited in step b - 1)
+            if (!warp_wait(ab, &sm.step_full[(b + 2) % NSTG], (uint32_t)((b + 2) / NSTG) & 1u)) break;
             tc_fence_after();
             g1a(b + 1);
         }
@@ -697,7 +644,6 @@ __device__ void s_role(SpSmem& sm, const SpCtx& x, int warp, int lane, const flo
     const int q = warp & 3, ch = warp >> 2;
     const int k = 32 * q + lane;  // dk row
     const int j0 = 24 * ch;       // first of this thread's 24 columns
-    STAMP_INIT;
     const uint32_t tl = x.tmem + lane_base(warp);
     constexpr uint32_t LO = NT * DK * 2;
     const size_t srow = (((size_t)x.s * x.Hv + x.h) * DK + k) * DV + x.col0 + j0;
@@ -719,7 +665,6 @@ __device__ void s_role(SpSmem& sm, const SpCtx& x, int warp, int lane, const flo
         const float gam = gam_next;
         if (b + 1 < x.n) gam_next = x.vec(b + 1)[rec::VEC_GAMMA];
         if (!warp_wait(&sm.abort, &sm.acc3_full, (uint32_t)b & 1u)) { ok = false; break; }
-        if (warp == 0) STAMP(b, 10);
         tc_fence_after();
         float v[24];
         ld_sum24(tl + T_ACC3 + j0, v);
@@ -730,7 +675,6 @@ __device__ void s_role(SpSmem& sm, const SpCtx& x, int warp, int lane, const flo
             fence_async_smem();
         }
         tc_fence_before();
-        if (warp == 0) STAMP(b, 11);
         mbar_arrive(&sm.s_ready);
     }
     if (ok && final_state && *(volatile int*)&sm.abort == 0) {
@@ -748,7 +692,6 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
     const int r = 16 * q + lane;  // accumulator row (valid for lane < 16)
     const int j0 = 24 * ch;
     const uint32_t tl = x.tmem + lane_base(warp);
-    STAMP_INIT;
     // per-chunk scalars, loaded a step before their use
     float gam_next = 1.f, d_next = lane < 16 ? x.vec(0)[rec::VEC_D + r] : 0.f;
     for (int b = -1; b + 1 < x.n; ++b) {
@@ -760,7 +703,6 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
             d_next = lane < 16 ? x.vec(b + 2)[rec::VEC_D + r] : 0.f;
         }
         if (!warp_wait(&sm.abort, &sm.acc1_full[x1], (uint32_t)((b + 1) >> 1) & 1u)) return;
-        if (warp == 8) STAMP(b + 1, 12);
         tc_fence_after();
         float v[24];
         ld_sum24(tl + T_ACC1 + 96 * x1 + j0, v);
@@ -769,12 +711,9 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
         if (lane < 16) put24(sm.y_op, OPB, r, 3 * ch, C, v);
         fence_async_smem();
         tc_fence_before();
-        if (warp == 8) STAMP(b + 1, 13);
         mbar_arrive(&sm.y_ready);
-        mbar_arrive(&sm.acc1_free[x1]);
         // Delta_{b+1} = -acc2 rows 0-31; D Delta_{b+1}
         if (!warp_wait(&sm.abort, &sm.acc2_full[x1], (uint32_t)((b + 1) >> 1) & 1u)) return;
-        if (warp == 8) STAMP(b + 1, 14);
         tc_fence_after();
         ld_sum24(tl + T_ACC2 + 96 * x1 + j0, v);
         float w[24];
@@ -790,9 +729,7 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
         }
         fence_async_smem();
         tc_fence_before();
-        if (warp == 8) STAMP(b + 1, 15);
         mbar_arrive(&sm.d_ready);
-        mbar_arrive(&sm.acc2_free[x1]);
     }
 }
 
@@ -801,12 +738,11 @@ __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __
     const int q = warp & 3, ch = (warp - 8) >> 2;
     const int i = 16 * (q - 2) + lane;  // chunk position (valid for lane < 16)
     const int j0 = 24 * ch;
-    STAMP_INIT;
     const uint32_t tl = x.tmem + lane_base(warp);
     const int nvalid = DV - (x.col0 + j0);
-    // step -1 produces no output; its accumulators are released at once
-    mbar_arrive(&sm.acc1_free[0]);
-    mbar_arrive(&sm.acc2_free[0]);
+    // step -1 produces no output: its share of y_ready / d_ready phase 0 is given at once
+    mbar_arrive(&sm.y_ready);
+    mbar_arrive(&sm.d_ready);
     float e_next = lane < 16 ? x.vec(0)[rec::VEC_E + i] : 0.f;  // loaded a step ahead
     for (int b = 0; b < x.n; ++b) {
         const int x1 = (b + 1) & 1;
@@ -818,13 +754,13 @@ __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __
         float qs[24];
         ld_sum24(tl + T_ACC1 + 96 * x1 + j0, qs);
         tc_fence_before();
-        mbar_arrive(&sm.acc1_free[x1]);
+        mbar_arrive(&sm.y_ready);
         if (!warp_wait(&sm.abort, &sm.acc2_full[x1], ph)) return;
         tc_fence_after();
         float pd[24];
         ld_sum24(tl + T_ACC2 + 96 * x1 + j0, pd);
         tc_fence_before();
-        mbar_arrive(&sm.acc2_free[x1]);
+        mbar_arrive(&sm.d_ready);
         const long long c0 = x.t0 + (long long)b * C;
         if (lane < 16 && c0 + i < x.t1) {
             float* op = out + ((size_t)(c0 + i) * x.Hv + x.h) * DV + x.col0 + j0;
@@ -875,23 +811,17 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (tid == 0) {
         for (int i = 0; i < NSTG; ++i) {
-            mbar_init(&sm.kq_full[i], 1);
-            mbar_init(&sm.kq_empty[i], 1);
-            mbar_init(&sm.v_full[i], 1);
-            mbar_init(&sm.v_empty[i], 1);
-            mbar_init(&sm.slot_full[i], 1);
-            mbar_init(&sm.slot_empty[i], 1);
+            mbar_init(&sm.step_full[i], 1);
+            mbar_init(&sm.step_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.acc1_full[i], 1);
             mbar_init(&sm.acc2_full[i], 1);
-            mbar_init(&sm.acc1_free[i], 256);
-            mbar_init(&sm.acc2_free[i], 256);
         }
         mbar_init(&sm.acc3_full, 1);
         mbar_init(&sm.s_ready, 256);
-        mbar_init(&sm.y_ready, 128);
-        mbar_init(&sm.d_ready, 128);
+        mbar_init(&sm.y_ready, 256);  // Y warps and output warps
+        mbar_init(&sm.d_ready, 256);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         mbar_init_fence();
@@ -1017,9 +947,6 @@ cudaError_t launch_prefill_tc(const FwdParams& p, cudaStream_t stream) {
     return e != cudaSuccess ? e : f;
 }
 
-#ifdef GDR_TC_STAMP
-void set_stamp_buffer(long long* p) { cudaMemcpyToSymbol(g_stamp, &p, sizeof(p)); }
-#endif
 
 int read_and_clear_tc_status() {
     int v = 0;

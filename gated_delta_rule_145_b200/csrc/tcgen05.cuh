@@ -108,24 +108,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test for completion of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity; false if it did not complete in time.
-// Out of line: one copy of the polling loop serves every call site, which keeps the
-// kernels' code small (code that is not resident in the instruction cache costs far more
-// than the call).
+// Polls with the non-blocking test and a short sleep between polls: blocking try_wait
+// instructions held by many waiting warps at once congest the shared-memory pipe and slow
+// every other warp's shared-memory, mbarrier and tensor-core traffic.  The polling loop
+// is out of line (one copy serves every call site).
 __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity);
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test(bar, parity)) return true;
     return mbar_wait_slow(bar, parity);
 }
 __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer();
-    // kept rolled: every call site inlines this loop, and an unrolled copy per site
-    // would swell the kernels past the instruction cache
     for (;;) {
 #pragma unroll 1
         for (int i = 0; i < 64; ++i) {
-            if (mbar_try_wait(bar, parity)) return true;
-            __nanosleep(kPollSleepNs);  // leave the issue slots to the working warps
+            __nanosleep(kPollSleepNs);
+            if (mbar_test(bar, parity)) return true;
         }
         if (globaltimer() - t0 > kWaitLimitNs) return false;
     }
