@@ -372,7 +372,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 constexpr int NT = 48;                      // dv columns per CTA
 constexpr int NTILES = (DV + NT - 1) / NT;  // 3 (the last a third empty)
 constexpr int NSTG = 3;                     // ring depth of tiles and records
-constexpr int SP_THREADS = 576;             // 18 warps
+constexpr int SP_THREADS = 640;             // 20 warps
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t T_ACC1 = 0;    // 2 x 96, M = 64: [K_{c+1}; Q_c] [S_hi | S_lo]
 constexpr uint32_t T_ACC2 = 192;  // 2 x 96, M = 64: rows 0-31 -Delta_{c+1}, 32-63 P_c Delta_c
@@ -384,8 +384,11 @@ constexpr uint32_t OPB = NT * C * 2;  // one K = 32 x N = 48 bf16 operand part (
 //          24 columns per warp half) and the state's hi/lo operand
 //   8, 9, 12, 13   Y and Delta epilogues (accumulator rows 0-31)
 //   10, 11, 14, 15 output epilogue (accumulator rows 32-63)
-//   16     tensor-core issue (one lane)
 //   17     loads: TMA tiles and record images (one lane)
+//   18     tensor-core issue of the Delta chain: U, [M;P] Delta, Wt Y (one lane)
+//   19     tensor-core issue of the state path: K^T D Delta and [K;Q] S (one lane)
+//   16     no role (it places warps 18 and 19 on sub-partitions 2 and 3, beside the
+//          small S and output code)
 struct alignas(1024) SpSmem {
     // pair buffer b: per dk half (8 KB) rows 0-31 K_{b+1}, rows 32-63 Q_b; 128-byte swizzle
     uint8_t kq[NSTG][16384];
@@ -397,16 +400,21 @@ struct alignas(1024) SpSmem {
     } slot[NSTG];
     // thread-written MN-major no-swizzle B operands, hi part then lo part along N
     uint8_t s_op[2 * NT * DK * 2];  // S: K = 128
-    uint8_t y_op[2 * OPB];          // Y
+    uint8_t y_op[2][2 * OPB];       // Y (two buffers)
     uint8_t d_op[2][2 * OPB];       // Delta (two buffers)
     uint8_t dd_op[2][2 * OPB];      // diag(D) Delta
     // step b's loads (pair b, V_{b+1}, record operands of step b) share ring entry
     // (b + 1) % NSTG and one full / one empty barrier
     uint64_t step_full[NSTG], step_empty[NSTG];
     uint64_t acc1_full[2], acc2_full[2], acc3_full;
-    // s_ready: S group wrote S_{b+1}.  y_ready: Y_{b+1} written and acc1 of step b read.
-    // d_ready: Delta_{b+1} written and acc2 of step b read.
-    uint64_t s_ready, y_ready, d_ready, drain;
+    // Every barrier below can complete its next phase only after each of its waiters has
+    // passed the current one, which keeps parity waits unambiguous:
+    //   s_ready       S group wrote S_{b+1}                         (state warp waits)
+    //   y_ready[x]    Y_{b+1} written to y_op[x], x = (b+1) & 1     (chain warp)
+    //   acc1_free[x]  acc1[x] read by the Y and output epilogues    (state warp)
+    //   d_ready       Delta_{b+1} written, acc2 of step b read      (chain warp)
+    //   dd_ready[x]   D Delta_{b+1} written to dd_op[x]             (state warp)
+    uint64_t s_ready, y_ready[2], acc1_free[2], d_ready, dd_ready[2], drain, drain2;
     uint32_t tmem_base;
     int abort;
 };
@@ -519,22 +527,100 @@ __device__ void load_role(SpSmem& sm, const SpCtx& x, int lane, const CUtensorMa
     __syncwarp();
 }
 
-// ----------------------------------------------------------- tensor-core issue (warp 16)
-__device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
+// ----------------------------------------------------------- tensor-core issue
+// Two issuing warps: the Delta chain (acc2) and the state path (acc3, acc1).  Each commit
+// covers only its own warp's products; the orderings that cross warps are noted below.
+
+// Delta chain, warp 18.  Step b: acc2 = U_{b+1} + [M_{b+1}; P_b] Delta_b + Wt_{b+1} Y_{b+1}.
+__device__ void chain_role(SpSmem& sm, const SpCtx& x, int lane) {
     const uint32_t id96 = idesc_bf16(64, 2 * NT, 0, 1);
     const uint32_t id48 = idesc_bf16(64, NT, 0, 1);
-    const uint32_t id_g3 = idesc_bf16(128, 2 * NT, 1, 1);
-    const uint64_t d_kq = sdesc(smem_u32(sm.kq[0]), 16, 1024, kSw128);    // [K;Q] K-major
-    const uint64_t d_kt = sdesc(smem_u32(sm.kq[0]), 8192, 1024, kSw128);  // K^T MN-major
     const uint64_t d_vt = sdesc(smem_u32(sm.vt[0]), 8192, 1024, kSw128);  // V MN-major
-    const uint64_t d_s = sdesc(smem_u32(sm.s_op), 128, 2048, kSwNone);
-    const uint64_t d_y = sdesc(smem_u32(sm.y_op), 128, 512, kSwNone);
+    const uint64_t d_y = sdesc(smem_u32(sm.y_op[0]), 128, 512, kSwNone);
     const uint64_t d_d = sdesc(smem_u32(sm.d_op[0]), 128, 512, kSwNone);
-    const uint64_t d_dd = sdesc(smem_u32(sm.dd_op[0]), 128, 512, kSwNone);
     const uint64_t d_wt = sdesc(smem_u32(sm.slot[0].wt[0]), 128, 512, kSwNone);
     const uint64_t d_ntb = sdesc(smem_u32(sm.slot[0].ntb[0]), 128, 512, kSwNone);
     const uint64_t d_mp = sdesc(smem_u32(sm.slot[0].mp[0]), 128, 512, kSwNone);
     constexpr uint32_t SLOT = sizeof(SpSmem::Slot);
+    constexpr uint32_t DBUF = 2 * OPB;
+    const bool leader = lane == 0;
+    int* ab = &sm.abort;
+    for (int b = -1; b < x.n; ++b) {
+        const int r = (b + 1) % NSTG, use = (b + 1) / NSTG;
+        const int x2 = (b + 1) & 1;
+        const uint32_t t2 = x.tmem + T_ACC2 + 96 * x2;
+        const bool nd = b + 1 < x.n;  // Delta_{b+1} needed
+        // acc2[x2] was last read in step b - 2: d_ready phase b - 1, waited in step b - 1
+        if (!warp_wait(ab, &sm.step_full[r], (uint32_t)use & 1u)) break;
+        tc_fence_after();
+        if (nd) {
+            // U: [-Tb_{b+1}; 0] (hi -> columns 0-47, lo -> 48-95) V_{b+1}
+            if (leader) {
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                        mma_bf16(t2 + NT * part, dadd(d_ntb, r * SLOT + part * 4096 + ks * 256),
+                                 dadd(d_vt, r * 4096 + ks * 2048), id48, ks > 0);
+            }
+            __syncwarp();
+        }
+        if (b >= 0) {
+            if (!warp_wait(ab, &sm.d_ready, (uint32_t)b & 1u)) break;  // Delta_b
+            tc_fence_after();
+            if (leader) {
+                // [M_{b+1}; P_b] Delta_b
+                const uint64_t bd = dadd(d_d, (b & 1) * DBUF);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(t2, dadd(d_mp, r * SLOT + ks * 256), dadd(bd, ks * 256), id96,
+                             nd ? 1u : (uint32_t)(ks > 0));
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(t2, dadd(d_mp, r * SLOT + 4096 + ks * 256), dadd(bd, ks * 256), id48, 1);
+            }
+            __syncwarp();
+        }
+        if (nd) {
+            // Y_{b+1}
+            if (!warp_wait(ab, &sm.y_ready[(b + 1) & 1], (uint32_t)((b + 1) >> 1) & 1u)) break;
+            tc_fence_after();
+            if (leader) {
+                const uint64_t by = dadd(d_y, ((b + 1) & 1) * DBUF);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(t2, dadd(d_wt, r * SLOT + ks * 256), dadd(by, ks * 256), id96, 1);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(t2, dadd(d_wt, r * SLOT + 4096 + ks * 256), dadd(by, ks * 256), id48, 1);
+            }
+            __syncwarp();
+        }
+        if (leader) {
+            mma_commit(&sm.acc2_full[x2]);
+            mma_commit(&sm.step_empty[r]);  // this warp is done with step b's V and operands
+        }
+        __syncwarp();
+    }
+    // everything issued has completed before the CTA may exit
+    if (leader) {
+        mma_commit(&sm.drain);
+        mbar_wait(&sm.drain, 0);
+    }
+    __syncwarp();
+}
+
+// State path, warp 19.  Step b: acc3 = K_b^T [D Delta_b hi | lo], then G1a(b+1):
+// acc1 = [K_{b+2}; Q_{b+1}] [S_{b+1} hi | lo].  Y is double-buffered: Y-epi(b) follows
+// this warp's G1a(b), not the chain warp's G1b(b-1), so it writes the other buffer; the
+// buffer it overwrites was read by G1b(b-2), complete before acc2 of step b-2 fired.
+__device__ void state_mma_role(SpSmem& sm, const SpCtx& x, int lane) {
+    const uint32_t id96 = idesc_bf16(64, 2 * NT, 0, 1);
+    const uint32_t id_g3 = idesc_bf16(128, 2 * NT, 1, 1);
+    const uint64_t d_kq = sdesc(smem_u32(sm.kq[0]), 16, 1024, kSw128);    // [K;Q] K-major
+    const uint64_t d_kt = sdesc(smem_u32(sm.kq[0]), 8192, 1024, kSw128);  // K^T MN-major
+    const uint64_t d_s = sdesc(smem_u32(sm.s_op), 128, 2048, kSwNone);
+    const uint64_t d_dd = sdesc(smem_u32(sm.dd_op[0]), 128, 512, kSwNone);
     constexpr uint32_t DBUF = 2 * OPB;
     const bool leader = lane == 0;
     int* ab = &sm.abort;
@@ -555,43 +641,14 @@ __device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
 
     if (!warp_wait(ab, &sm.s_ready, 0)) goto drain;  // S_0 in place
     if (!warp_wait(ab, &sm.step_full[0], 0)) goto drain;
+    tc_fence_after();
     g1a(-1);
     for (int b = -1; b < x.n; ++b) {
-        const int r = (b + 1) % NSTG, use = (b + 1) / NSTG;
-        const int x2 = (b + 1) & 1;
-        const uint32_t t2 = x.tmem + T_ACC2 + 96 * x2;
-        const bool nd = b + 1 < x.n;  // Delta_{b+1} needed
-        // acc2[x2] was last read in step b - 2, covered by d_ready phase b - 1 (waited in
-        // step b - 1)
-        if (!warp_wait(ab, &sm.step_full[r], (uint32_t)use & 1u)) break;
-        tc_fence_after();
-        bool first = true;
-        if (nd) {
-            // U: [-Tb_{b+1}; 0] (hi -> columns 0-47, lo -> 48-95) V_{b+1}
-            if (leader) {
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks)
-                        mma_bf16(t2 + NT * part, dadd(d_ntb, r * SLOT + part * 4096 + ks * 256),
-                                 dadd(d_vt, r * 4096 + ks * 2048), id48, ks > 0);
-            }
-            __syncwarp();
-            first = false;
-        }
         if (b >= 0) {
-            if (!warp_wait(ab, &sm.d_ready, (uint32_t)b & 1u)) break;  // Delta_b, D Delta_b
+            // acc3 was read by S-epi(b - 1) before s_ready phase b, waited before G1a(b)
+            if (!warp_wait(ab, &sm.dd_ready[b & 1], (uint32_t)(b >> 1) & 1u)) break;  // D Delta_b
             tc_fence_after();
             if (leader) {
-                const uint64_t bd = dadd(d_d, (b & 1) * DBUF);
-                // [M_{b+1}; P_b] Delta_b
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-                    mma_bf16(t2, dadd(d_mp, r * SLOT + ks * 256), dadd(bd, ks * 256), id96,
-                             first ? (ks > 0) : 1);
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-                    mma_bf16(t2, dadd(d_mp, r * SLOT + 4096 + ks * 256), dadd(bd, ks * 256), id48, 1);
                 // acc3 = K_b^T [D Delta_b hi | lo]   (K_b sits in pair buffer b - 1)
                 const uint64_t bdd = dadd(d_dd, (b & 1) * DBUF);
 #pragma unroll
@@ -599,31 +656,15 @@ __device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
                     mma_bf16(x.tmem + T_ACC3, dadd(d_kt, (b % NSTG) * 16384 + ks * 2048),
                              dadd(bdd, ks * 256), id_g3, ks > 0);
                 mma_commit(&sm.acc3_full);
-                mma_commit(&sm.step_empty[b % NSTG]);  // step b - 1's loads all read
+                mma_commit(&sm.step_empty[b % NSTG]);  // pair buffer b - 1 read for the last time
             }
             __syncwarp();
         }
-        if (nd) {
-            if (!warp_wait(ab, &sm.y_ready, (uint32_t)(b + 1) & 1u)) break;  // Y_{b+1}
-            tc_fence_after();
-            if (leader) {
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-                    mma_bf16(t2, dadd(d_wt, r * SLOT + ks * 256), dadd(d_y, ks * 256), id96, 1);
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-                    mma_bf16(t2, dadd(d_wt, r * SLOT + 4096 + ks * 256), dadd(d_y, ks * 256), id48, 1);
-            }
-            __syncwarp();
-        }
-        if (leader) {
-            mma_commit(&sm.acc2_full[x2]);
-        }
-        __syncwarp();
-        if (nd) {
-            // G1a(b+1) needs S_{b+1} (phase b + 1 of s_ready) and a free acc1 buffer
-            if (b >= 0 && !warp_wait(ab, &sm.s_ready, (uint32_t)(b + 1) & 1u)) break;
-            // acc1 of step b - 1 was read before y_ready phase b (waited in step b - 1)
+        if (b + 1 < x.n) {
+            // G1a(b+1): S_{b+1} (s_ready phase b + 1); acc1[b & 1] read after G1a(b - 1)
+            // (its use b >> 1); pair b + 1 loaded
+            if (!warp_wait(ab, &sm.s_ready, (uint32_t)(b + 1) & 1u)) break;
+            if (b >= 0 && !warp_wait(ab, &sm.acc1_free[b & 1], (uint32_t)(b >> 1) & 1u)) break;
             if (!warp_wait(ab, &sm.step_full[(b + 2) % NSTG], (uint32_t)((b + 2) / NSTG) & 1u)) break;
             tc_fence_after();
             g1a(b + 1);
@@ -632,8 +673,8 @@ __device__ void mma_role(SpSmem& sm, const SpCtx& x, int lane) {
 drain:
     // everything issued has completed before the CTA may exit
     if (leader) {
-        mma_commit(&sm.drain);
-        mbar_wait(&sm.drain, 0);
+        mma_commit(&sm.drain2);
+        mbar_wait(&sm.drain2, 0);
     }
     __syncwarp();
 }
@@ -708,10 +749,11 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
         ld_sum24(tl + T_ACC1 + 96 * x1 + j0, v);
 #pragma unroll
         for (int j = 0; j < 24; ++j) v[j] *= gam;
-        if (lane < 16) put24(sm.y_op, OPB, r, 3 * ch, C, v);
+        if (lane < 16) put24(sm.y_op[(b + 1) & 1], OPB, r, 3 * ch, C, v);
         fence_async_smem();
         tc_fence_before();
-        mbar_arrive(&sm.y_ready);
+        mbar_arrive(&sm.y_ready[(b + 1) & 1]);
+        mbar_arrive(&sm.acc1_free[x1]);
         // Delta_{b+1} = -acc2 rows 0-31; D Delta_{b+1}
         if (!warp_wait(&sm.abort, &sm.acc2_full[x1], (uint32_t)((b + 1) >> 1) & 1u)) return;
         tc_fence_after();
@@ -730,6 +772,7 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.d_ready);
+        mbar_arrive(&sm.dd_ready[nb]);
     }
 }
 
@@ -740,8 +783,9 @@ __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __
     const int j0 = 24 * ch;
     const uint32_t tl = x.tmem + lane_base(warp);
     const int nvalid = DV - (x.col0 + j0);
-    // step -1 produces no output: its share of y_ready / d_ready phase 0 is given at once
-    mbar_arrive(&sm.y_ready);
+    // step -1 produces no output: its share of acc1_free[0] / d_ready phase 0 is given at
+    // once
+    mbar_arrive(&sm.acc1_free[0]);
     mbar_arrive(&sm.d_ready);
     float e_next = lane < 16 ? x.vec(0)[rec::VEC_E + i] : 0.f;  // loaded a step ahead
     for (int b = 0; b < x.n; ++b) {
@@ -754,7 +798,7 @@ __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __
         float qs[24];
         ld_sum24(tl + T_ACC1 + 96 * x1 + j0, qs);
         tc_fence_before();
-        mbar_arrive(&sm.y_ready);
+        mbar_arrive(&sm.acc1_free[x1]);
         if (!warp_wait(&sm.abort, &sm.acc2_full[x1], ph)) return;
         tc_fence_after();
         float pd[24];
@@ -812,7 +856,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid == 0) {
         for (int i = 0; i < NSTG; ++i) {
             mbar_init(&sm.step_full[i], 1);
-            mbar_init(&sm.step_empty[i], 1);
+            mbar_init(&sm.step_empty[i], 2);  // released by both issuing warps
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.acc1_full[i], 1);
@@ -820,9 +864,14 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         mbar_init(&sm.acc3_full, 1);
         mbar_init(&sm.s_ready, 256);
-        mbar_init(&sm.y_ready, 256);  // Y warps and output warps
-        mbar_init(&sm.d_ready, 256);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.y_ready[i], 128);    // Y warps
+            mbar_init(&sm.acc1_free[i], 256);  // Y warps and output warps
+            mbar_init(&sm.dd_ready[i], 128);   // Delta warps
+        }
+        mbar_init(&sm.d_ready, 256);           // Delta warps and output warps
         mbar_init(&sm.drain, 1);
+        mbar_init(&sm.drain2, 1);
         sm.abort = 0;
         mbar_init_fence();
         tma_prefetch_map(&tm_q);
@@ -847,10 +896,12 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         s_role(sm, x, warp, lane, init_state, final_state);
     else if (warp < 16)
         ((warp & 3) < 2) ? d_role(sm, x, warp, lane) : o_role(sm, x, warp, lane, out);
-    else if (warp == 16)
-        mma_role(sm, x, lane);
-    else
+    else if (warp == 17)
         load_role(sm, x, lane, &tm_q, &tm_k, &tm_v);
+    else if (warp == 18)
+        chain_role(sm, x, lane);
+    else if (warp == 19)
+        state_mma_role(sm, x, lane);
 
     tc_fence_before();
     __syncthreads();
