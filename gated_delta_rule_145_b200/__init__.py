@@ -31,6 +31,7 @@ GDR_ERR_ALIGN = -4
 GDR_ERR_OOM = -5
 GDR_ERR_CUDA = -6
 GDR_ERR_TIMEOUT = -7
+GDR_ERR_TOO_LARGE = -8
 
 
 class GdrError(RuntimeError):
@@ -46,6 +47,7 @@ _I = ctypes.c_int
 _SIGS = {
     "gdr_prefill_chunked": [_P] * 11 + [_I] * 7 + [_P],
     "gdr_prefill_chunked_f32": [_P] * 11 + [_I] * 7 + [_P],
+    "gdr_prefill_chunked_noalloc": [_P] * 11 + [_I] * 7 + [_P],
     "gdr_prefill_recurrent": [_P] * 11 + [_I] * 6 + [_P],
     "gdr_prefill_recurrent_f32": [_P] * 11 + [_I] * 6 + [_P],
     "gdr_decode_step": [_P] * 9 + [_I] * 5 + [_P],
@@ -118,6 +120,15 @@ def _call(name, ptrs, ints, stream, check):
 def gdr_prefill_chunked(q, k, v, a, b, A_log, dt_bias, init_state, out, final_state, cu_seqlens,
                         B, T, Hk, Hv, dk, dv, chunk, stream=None, check=True):
     return _call("gdr_prefill_chunked",
+                 (q, k, v, a, b, A_log, dt_bias, init_state, out, final_state, cu_seqlens),
+                 (B, T, Hk, Hv, dk, dv, chunk), stream, check)
+
+
+def gdr_prefill_chunked_noalloc(q, k, v, a, b, A_log, dt_bias, init_state, out, final_state,
+                                cu_seqlens, B, T, Hk, Hv, dk, dv, chunk, stream=None, check=True):
+    """gdr_prefill_chunked on the library's fixed scratch: no device memory is allocated
+    (bf16, dk = dv = 128, chunk 32; see include/gdr.h for the size limit)."""
+    return _call("gdr_prefill_chunked_noalloc",
                  (q, k, v, a, b, A_log, dt_bias, init_state, out, final_state, cu_seqlens),
                  (B, T, Hk, Hv, dk, dv, chunk), stream, check)
 

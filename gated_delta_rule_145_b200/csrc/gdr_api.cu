@@ -96,6 +96,22 @@ int gdr_prefill_chunked(const void* q, const void* k, const void* v, const void*
                            (cudaStream_t)stream);
 }
 
+int gdr_prefill_chunked_noalloc(const void* q, const void* k, const void* v, const void* a,
+                                const void* b, const float* A_log, const float* dt_bias,
+                                const float* init_state, float* out, float* final_state,
+                                const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                                int dv, int chunk, gdr_stream_t stream) {
+    const FwdParams p = make_params(q, k, v, a, b, A_log, dt_bias, init_state, out, final_state,
+                                    cu_seqlens, B, T, Hk, Hv, dk, dv, chunk, InType::BF16);
+    const int rc = check_common(p, 2);
+    if (rc != GDR_OK) return rc;
+    if (p.chunk != 32 || p.dk != 128 || p.dv != 128 || p.T < 1) return GDR_ERR_UNSUPPORTED;
+    if (gdr::prefill_tc_workspace_bytes(p) > gdr::noalloc_scratch_bytes()) return GDR_ERR_TOO_LARGE;
+    void* ws = nullptr;
+    if (gdr::noalloc_scratch(&ws) != cudaSuccess) return GDR_ERR_CUDA;
+    return to_status(gdr::launch_prefill_tc_ws(p, ws, (cudaStream_t)stream));
+}
+
 int gdr_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,
                             const float* b, const float* A_log, const float* dt_bias,
                             const float* init_state, float* out, float* final_state,
@@ -162,6 +178,9 @@ const char* gdr_status_string(int status) {
         case GDR_ERR_OOM: return "GDR_ERR_OOM: the prefill workspace could not be allocated";
         case GDR_ERR_CUDA: return "GDR_ERR_CUDA: kernel launch failed";
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a kernel abandoned a bounded wait";
+        case GDR_ERR_TOO_LARGE:
+            return "GDR_ERR_TOO_LARGE: the call needs more workspace than the fixed 64 MiB scratch "
+                   "of gdr_prefill_chunked_noalloc";
         default: return "unknown status";
     }
 }

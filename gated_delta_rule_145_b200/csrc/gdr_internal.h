@@ -40,6 +40,11 @@ cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stre
 // Returns the cached workspace memory of every device to the system; prefill_tc.cu.
 void workspace_release();
 
+// The fixed scratch area of the no-allocation prefill entry point: its size, and its
+// device address on the current device (looked up once per device); noalloc.cu.
+size_t noalloc_scratch_bytes();
+cudaError_t noalloc_scratch(void** ptr);
+
 // Reads and clears the tensor-core kernels' timeout record (nonzero if set, 0 if not,
 // -1 on a CUDA error); prefill_tc.cu.
 int read_and_clear_tc_status();

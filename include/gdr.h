@@ -68,6 +68,7 @@ typedef void* gdr_stream_t; /* cudaStream_t */
 #define GDR_ERR_OOM (-5)         /* the prefill workspace could not be allocated */
 #define GDR_ERR_CUDA (-6)        /* a kernel launch failed */
 #define GDR_ERR_TIMEOUT (-7)     /* a kernel gave up a bounded on-chip wait (see below) */
+#define GDR_ERR_TOO_LARGE (-8)   /* more workspace than gdr_prefill_chunked_noalloc's scratch */
 
 /*
  * Chunked (UT-transform) prefill.  Source: Mila "GatedDeltaRule.ixx File Reference",
@@ -93,6 +94,38 @@ GDR_API int gdr_prefill_chunked(const void* q, const void* k, const void* v, con
                         const float* init_state, float* out, float* final_state,
                         const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
                         int dv, int chunk, gdr_stream_t stream);
+
+/*
+ * gdr_prefill_chunked without any memory allocation, for callers that cannot allocate
+ * device memory during a call: for example a host framework whose own caching allocator
+ * already owns the device memory, or a latency-critical path where an allocation (which
+ * may synchronise the device, or fail when memory is fragmented) is not acceptable.
+ * The pages have no counterpart for this call: it only changes where the prefill keeps
+ * its intermediate records.
+ *
+ * Same arguments, layouts and results as gdr_prefill_chunked, restricted to bf16 inputs
+ * with dk = dv = 128, chunk = 32 and T >= 1 (anything else returns GDR_ERR_UNSUPPORTED;
+ * use gdr_prefill_chunked there).  Instead of a pooled workspace the call uses a fixed
+ * 64 MiB scratch array compiled into the library, which every device that loads the
+ * library holds until the process exits.  The workspace needed is 16896 bytes per
+ * (chunk, value head) -- dense mode B * ceil(T / 32) * Hv records, varlen mode at most
+ * ((T + 31 B) / 32 + 1) * Hv -- so at most 3971 records fit (e.g. T = 2560 at Hv = 48);
+ * larger calls return GDR_ERR_TOO_LARGE before anything is enqueued.  It calls no
+ * allocator (no cudaMalloc, cudaMallocAsync or cudaFree).
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ *     capture on the device.
+ *   - Every call on a device shares the same scratch.  The call writes every record it
+ *     reads, so nothing needs to start at zero and later calls see no stale state; but
+ *     calls that overlap on the GPU (on different streams without ordering between
+ *     them) race on the scratch and must not be issued.
+ */
+GDR_API int gdr_prefill_chunked_noalloc(const void* q, const void* k, const void* v,
+                                        const void* a, const void* b, const float* A_log,
+                                        const float* dt_bias, const float* init_state,
+                                        float* out, float* final_state,
+                                        const int32_t* cu_seqlens, int B, int T, int Hk,
+                                        int Hv, int dk, int dv, int chunk, gdr_stream_t stream);
 
 /* As gdr_prefill_chunked with fp32 q, k, v, a, b. */
 GDR_API int gdr_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,
