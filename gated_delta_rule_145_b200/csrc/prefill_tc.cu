@@ -103,18 +103,27 @@ __device__ __forceinline__ float sumsq64(const uint8_t* line) {
     return s0 + s1;
 }
 
-// Row m of a 32 x 32 operand image (hi and lo parts): sgn * src[0..31].
-__device__ __forceinline__ void store_image_row(const float* __restrict__ src, float sgn,
+// Row m of a 32 x 32 operand image (hi and lo parts): sgn * src[j] * cs[j] (cs may be
+// null: no column scale).
+__device__ __forceinline__ void store_image_row(const float* __restrict__ src,
+                                                const float* __restrict__ cs, float sgn,
                                                 uint8_t* hi, uint8_t* lo, int m) {
 #pragma unroll
     for (int kc = 0; kc < 4; ++kc) {
-        const float4 s0 = *reinterpret_cast<const float4*>(src + 8 * kc);
-        const float4 s1 = *reinterpret_cast<const float4*>(src + 8 * kc + 4);
+        float4 s0 = *reinterpret_cast<const float4*>(src + 8 * kc);
+        float4 s1 = *reinterpret_cast<const float4*>(src + 8 * kc + 4);
+        float4 c0 = make_float4(sgn, sgn, sgn, sgn), c1 = c0;
+        if (cs) {
+            const float4 a0 = *reinterpret_cast<const float4*>(cs + 8 * kc);
+            const float4 a1 = *reinterpret_cast<const float4*>(cs + 8 * kc + 4);
+            c0 = make_float4(sgn * a0.x, sgn * a0.y, sgn * a0.z, sgn * a0.w);
+            c1 = make_float4(sgn * a1.x, sgn * a1.y, sgn * a1.z, sgn * a1.w);
+        }
         uint4 hv, lv;
-        split2(sgn * s0.x, sgn * s0.y, hv.x, lv.x);
-        split2(sgn * s0.z, sgn * s0.w, hv.y, lv.y);
-        split2(sgn * s1.x, sgn * s1.y, hv.z, lv.z);
-        split2(sgn * s1.z, sgn * s1.w, hv.w, lv.w);
+        split2(c0.x * s0.x, c0.y * s0.y, hv.x, lv.x);
+        split2(c0.z * s0.z, c0.w * s0.w, hv.y, lv.y);
+        split2(c1.x * s1.x, c1.y * s1.y, hv.z, lv.z);
+        split2(c1.z * s1.z, c1.w * s1.w, hv.w, lv.w);
         *reinterpret_cast<uint4*>(hi + rec::k_off(m, kc)) = hv;
         *reinterpret_cast<uint4*>(lo + rec::k_off(m, kc)) = lv;
     }
@@ -123,21 +132,32 @@ __device__ __forceinline__ void store_image_row(const float* __restrict__ src, f
 // =============================================================== intra-chunk kernel
 
 struct alignas(1024) PrepSmem {
-    // per dk half (12 KB): K_prev rows 0-31 | K rows 32-63 | Q rows 64-95, 128-byte rows,
-    // 128-byte swizzle.  Gram A = [K;Q] (rows 32-95), B = [K_prev;K] (rows 0-63).
-    uint8_t kq[2][12288];
-    // fp32 32 x 32 blocks, rows padded to 36 floats (16-byte rows, conflict-free vectors)
-    float Am[C][36];
-    float Pm[C][36];
-    float R3[C][36];  // diag(w) K K_prev^T diag(D_prev)
     union {
+        // per dk half (12 KB): K_prev rows 0-31 | K rows 32-63 | Q rows 64-95, 128-byte
+        // rows, 128-byte swizzle.  Gram A = [K;Q] (rows 32-95), B = [K_prev;K] (rows 0-63).
+        // Dead once the Gram product and the norms are done; the fp32 blocks below reuse
+        // the space (a CTA of ~31 KB lets six run per SM).
+        uint8_t kq[2][12288];
         struct {
-            float KK[C][36];  // K K^T
-            float KR[C][36];  // K K_prev^T
-            float QK[C][36];  // Q K^T
-        } g;
-        float X[C][100];  // [Wt | Tb | M]
-    } u;
+            // fp32 32 x 32 blocks, rows padded to 36 floats (16-byte rows, conflict-free
+            // vectors)
+            union {
+                struct {
+                    float KK[C][36];  // K K^T
+                    float KR[C][36];  // K K_prev^T
+                    float QK[C][36];  // Q K^T
+                } g;
+                struct {
+                    float Tm[C][36];   // T = (I + A)^-1
+                    float Mm[C][36];   // M = T R3
+                    float Zm[16][20];  // A21 T11 (blocked inverse)
+                } t;
+            } u;
+            float Am[C][36];
+            float Pm[C][36];
+        } f;
+    };
+    float R3[C][36];  // diag(w) K K_prev^T diag(D_prev)
     alignas(16) float beta[C];
     alignas(16) float G[C];
     alignas(16) float eG[C];
@@ -150,10 +170,11 @@ struct alignas(1024) PrepSmem {
     uint64_t bar_tma, bar_mma;
     uint32_t tmem;
 };
+static_assert(sizeof(PrepSmem) <= 32 * 1024, "six intra-chunk CTAs per SM");
 
 constexpr int PREP_THREADS = 128;
 
-__global__ void __launch_bounds__(PREP_THREADS)
+__global__ void __launch_bounds__(PREP_THREADS, 6)
 intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                    const float* __restrict__ A_log, const float* __restrict__ dt_bias,
@@ -264,8 +285,8 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tmem_ld_wait();
         if (lane < 16) {
             const int r = 16 * warp + lane;
-            float* d0 = r < 32 ? sm.u.g.KR[r] : nullptr;
-            float* d1 = r < 32 ? sm.u.g.KK[r] : sm.u.g.QK[r - 32];
+            float* d0 = r < 32 ? sm.f.u.g.KR[r] : nullptr;
+            float* d1 = r < 32 ? sm.f.u.g.KK[r] : sm.f.u.g.QK[r - 32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 if (d0)
@@ -288,7 +309,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float* vec = reinterpret_cast<float*>(rc + rec::OFF_VEC);
     if (tid < C) {
         const int i = tid;
-        const float rk = inv_norm_fast(sm.u.g.KK[i][i]);
+        const float rk = inv_norm_fast(sm.f.u.g.KK[i][i]);
         sm.rk[i] = rk;
         sm.w[i] = sm.beta[i] * sm.eG[i] * rk;
         vec[rec::VEC_E + i] = sm.eG[i] * sm.rq[i];
@@ -310,60 +331,99 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int q = 0; q < 8; ++q) {
             const int j = j0 + q;
             const float dec = __expf(Gi - sm.G[j]) * sm.rk[j];  // used only where j <= i
-            am[q] = j < i ? fa * sm.u.g.KK[i][j] * dec : 0.f;
-            pm[q] = j <= i ? fp * sm.u.g.QK[i][j] * dec : 0.f;
-            r3[q] = wi * sm.u.g.KR[i][j] * sm.Dp[j];
+            am[q] = j < i ? fa * sm.f.u.g.KK[i][j] * dec : 0.f;
+            pm[q] = j <= i ? fp * sm.f.u.g.QK[i][j] * dec : 0.f;
+            r3[q] = wi * sm.f.u.g.KR[i][j] * sm.Dp[j];
         }
 #pragma unroll
         for (int q = 0; q < 8; q += 4) {
-            *reinterpret_cast<float4*>(&sm.Am[i][j0 + q]) = make_float4(am[q], am[q + 1], am[q + 2], am[q + 3]);
-            *reinterpret_cast<float4*>(&sm.Pm[i][j0 + q]) = make_float4(pm[q], pm[q + 1], pm[q + 2], pm[q + 3]);
+            *reinterpret_cast<float4*>(&sm.f.Am[i][j0 + q]) = make_float4(am[q], am[q + 1], am[q + 2], am[q + 3]);
+            *reinterpret_cast<float4*>(&sm.f.Pm[i][j0 + q]) = make_float4(pm[q], pm[q + 1], pm[q + 2], pm[q + 3]);
             *reinterpret_cast<float4*>(&sm.R3[i][j0 + q]) = make_float4(r3[q], r3[q + 1], r3[q + 2], r3[q + 3]);
         }
     }
     __syncthreads();
 
-    if (tid < 3 * C) {
-        // ---- forward substitution (I + A) x = rhs, one right-hand side per thread:
-        //      columns 0-31 diag(w), 32-63 diag(beta), 64-95 R3
-        const int mat = tid >> 5, jj = tid & 31;
-        float x[C];
+    // ---- T = (I + A)^-1 by 16 x 16 blocks.  Diagonal blocks by forward substitution,
+    //      one column per lane (lanes 0-15: T11, 16-31: T22; one short unrolled body), the
+    //      off-diagonal block as T21 = -T22 (A21 T11); strictly upper blocks are zero.
+    if (warp == 0) {
+        const int o = lane & 16, j = lane & 15;
+        float x[16];
 #pragma unroll
-        for (int i = 0; i < C; ++i) x[i] = 0.f;
+        for (int i = 0; i < 16; ++i) {
+            float s0 = i == j ? 1.f : 0.f, s1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            float bi;
-            if (mat == 0)
-                bi = i == jj ? sm.w[i] : 0.f;
-            else if (mat == 1)
-                bi = i == jj ? sm.beta[i] : 0.f;
-            else
-                bi = sm.R3[i][jj];
-            float s0 = bi, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-            for (int m = 0; m < (i & ~3); m += 4) {
-                const float4 av = *reinterpret_cast<const float4*>(&sm.Am[i][m]);
+            for (int m = 0; m < (i & ~1); m += 2) {
+                const float2 av = *reinterpret_cast<const float2*>(&sm.f.Am[o + i][o + m]);
                 s0 -= av.x * x[m];
                 s1 -= av.y * x[m + 1];
-                s2 -= av.z * x[m + 2];
-                s3 -= av.w * x[m + 3];
             }
-#pragma unroll
-            for (int m = i & ~3; m < i; ++m) s0 -= sm.Am[i][m] * x[m];
-            x[i] = (s0 + s1) + (s2 + s3);
+            if (i & 1) s0 -= sm.f.Am[o + i][o + i - 1] * x[i - 1];
+            x[i] = s0 + s1;
         }
 #pragma unroll
-        for (int i = 0; i < C; ++i) sm.u.X[i][tid] = x[i];
-    } else {
-        // ---- P image (warp 3, one row per lane)
-        store_image_row(sm.Pm[lane], 1.f, rc + rec::OFF_P, rc + rec::OFF_P + IMG, lane);
+        for (int i = 0; i < 16; ++i) {
+            sm.f.u.t.Tm[o + i][o + j] = x[i];
+            sm.f.u.t.Tm[i][16 + j] = 0.f;  // upper-right block (written twice, same value)
+        }
     }
     __syncthreads();
-    // ---- Wt, -Tb, M images: thread -> one row of one matrix
-    if (tid < 3 * C) {
+    {
+        // Z = A21 T11: thread -> row i, columns 2 cg, 2 cg + 1 (T11 lower triangular)
+        const int i = tid >> 3, j0 = 2 * (tid & 7);
+        float z0 = 0.f, z1 = 0.f;
+#pragma unroll 1
+        for (int m = 0; m < 16; ++m) {
+            const float a_ = sm.f.Am[16 + i][m];
+            z0 += a_ * sm.f.u.t.Tm[m][j0];
+            z1 += a_ * sm.f.u.t.Tm[m][j0 + 1];
+        }
+        sm.f.u.t.Zm[i][j0] = z0;
+        sm.f.u.t.Zm[i][j0 + 1] = z1;
+    }
+    __syncthreads();
+    {
+        // T21 = -T22 Z
+        const int i = tid >> 3, j0 = 2 * (tid & 7);
+        float t0 = 0.f, t1 = 0.f;
+#pragma unroll 1
+        for (int m = 0; m <= i; ++m) {
+            const float t_ = sm.f.u.t.Tm[16 + i][16 + m];
+            t0 += t_ * sm.f.u.t.Zm[m][j0];
+            t1 += t_ * sm.f.u.t.Zm[m][j0 + 1];
+        }
+        sm.f.u.t.Tm[16 + i][j0] = -t0;
+        sm.f.u.t.Tm[16 + i][j0 + 1] = -t1;
+    }
+    __syncthreads();
+    {
+        // M = T R3: thread -> row i, columns 8 cg .. 8 cg + 7 (T lower triangular)
+        const int i = tid >> 2, j0 = 8 * (tid & 3);
+        float mm[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mm[q] = 0.f;
+#pragma unroll 1
+        for (int m = 0; m <= i; ++m) {
+            const float t_ = sm.f.u.t.Tm[i][m];
+            const float4 r0 = *reinterpret_cast<const float4*>(&sm.R3[m][j0]);
+            const float4 r1 = *reinterpret_cast<const float4*>(&sm.R3[m][j0 + 4]);
+            mm[0] += t_ * r0.x; mm[1] += t_ * r0.y; mm[2] += t_ * r0.z; mm[3] += t_ * r0.w;
+            mm[4] += t_ * r1.x; mm[5] += t_ * r1.y; mm[6] += t_ * r1.z; mm[7] += t_ * r1.w;
+        }
+        *reinterpret_cast<float4*>(&sm.f.u.t.Mm[i][j0]) = make_float4(mm[0], mm[1], mm[2], mm[3]);
+        *reinterpret_cast<float4*>(&sm.f.u.t.Mm[i][j0 + 4]) = make_float4(mm[4], mm[5], mm[6], mm[7]);
+    }
+    __syncthreads();
+    // ---- the four operand images, one row of one matrix per thread:
+    //      Wt = T diag(w), -Tb = -T diag(beta), M, P
+    {
         const int mat = tid >> 5, i = tid & 31;
-        const uint32_t off = mat == 0 ? rec::OFF_WT : (mat == 1 ? rec::OFF_NTB : rec::OFF_M);
-        store_image_row(&sm.u.X[i][32 * mat], mat == 1 ? -1.f : 1.f, rc + off, rc + off + IMG, i);
+        const uint32_t off = mat == 0 ? rec::OFF_WT
+                                      : (mat == 1 ? rec::OFF_NTB : (mat == 2 ? rec::OFF_M : rec::OFF_P));
+        const float* src = mat < 2 ? sm.f.u.t.Tm[i] : (mat == 2 ? sm.f.u.t.Mm[i] : sm.f.Pm[i]);
+        const float* cs = mat == 0 ? sm.w : (mat == 1 ? sm.beta : nullptr);
+        store_image_row(src, cs, mat == 1 ? -1.f : 1.f, rc + off, rc + off + IMG, i);
     }
 }
 
