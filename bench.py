@@ -274,6 +274,17 @@ def bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth):
     # two kernels per call: intra-chunk, then state passing
     res = dict(inp=inp, region_ms=region_ms, launches=2 * args.steps,
                kernel_ms=statistics.mean(s.elapsed_time(e) for s, e in ev))
+    # the erase=False form (gated linear attention) on the same inputs and kernels
+    def gla(_i):
+        gdr.gdr_gla_prefill_chunked(q, k, v, a, b, A_log, dt_bias, None, out, fin, None,
+                                    P["B"], P["T"], P["Hk"], P["Hv"], P["dk"], P["dv"],
+                                    P["chunk"], stream=stream)
+
+    for i in range(3):
+        gla(i)
+    gla_steps = max(3, min(args.steps, 10))
+    res.update(gla_ms=_timed(dist, dev, stream, sampler, gla, gla_steps), gla_steps=gla_steps,
+               launches=res["launches"] + 2 * gla_steps)
     if args.no_e2e:
         return res
     # ---- end to end through the public API: pinned host inputs in, outputs back
@@ -398,6 +409,14 @@ def run_ours(args, dist):
                 "cpu_baseline": cpu,
             })
             result["gpu_launches"] += pre["launches"]
+            gla_s = pre["gla_ms"] / pre["gla_steps"] / 1e3
+            result["gla"] = {
+                "form": "erase=False (gated linear attention), same workload and kernels",
+                "value": round(P["B"] * P["T"] * dist.world / gla_s, 1), "unit": "tokens/s",
+                "ms_per_step": round(pre["gla_ms"] / pre["gla_steps"], 4),
+                "roofline": {"bound": "hbm", "achieved": round(alg_b / gla_s / 1e9, 1),
+                             "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(alg_b / gla_s / 1e9 / pk["hbm_gbs"], 4)}}
             if "e2e_ms" in pre:
                 result["e2e"] = {"value": round(P["B"] * P["T"] * pre["e2e_steps"] * dist.world /
                                                 (pre["e2e_ms"] / 1e3), 1),

@@ -52,6 +52,12 @@ _SIGS = {
     "gdr_prefill_recurrent_f32": [_P] * 11 + [_I] * 6 + [_P],
     "gdr_decode_step": [_P] * 9 + [_I] * 5 + [_P],
     "gdr_decode_step_f32": [_P] * 9 + [_I] * 5 + [_P],
+    "gdr_gla_prefill_chunked": [_P] * 11 + [_I] * 7 + [_P],
+    "gdr_gla_prefill_chunked_f32": [_P] * 11 + [_I] * 7 + [_P],
+    "gdr_gla_prefill_recurrent": [_P] * 11 + [_I] * 6 + [_P],
+    "gdr_gla_prefill_recurrent_f32": [_P] * 11 + [_I] * 6 + [_P],
+    "gdr_gla_decode_step": [_P] * 9 + [_I] * 5 + [_P],
+    "gdr_gla_decode_step_f32": [_P] * 9 + [_I] * 5 + [_P],
 }
 
 
@@ -185,12 +191,30 @@ def _check_tensors(tensors, dtype):
             raise ValueError(f"{name} must be {want}, got {t.dtype}")
 
 
+def _gla_wrapper(name, nptr):
+    """Mirror of the C entry point `name`: nptr pointer arguments, then the sizes."""
+    def fn(*args, stream=None, check=True):
+        return _call(name, args[:nptr], args[nptr:], stream, check)
+    fn.__name__ = name
+    fn.__doc__ = f"{name}: the erase=False (gated linear attention) form; see include/gdr.h."
+    return fn
+
+
+gdr_gla_prefill_chunked = _gla_wrapper("gdr_gla_prefill_chunked", 11)
+gdr_gla_prefill_chunked_f32 = _gla_wrapper("gdr_gla_prefill_chunked_f32", 11)
+gdr_gla_prefill_recurrent = _gla_wrapper("gdr_gla_prefill_recurrent", 11)
+gdr_gla_prefill_recurrent_f32 = _gla_wrapper("gdr_gla_prefill_recurrent_f32", 11)
+gdr_gla_decode_step = _gla_wrapper("gdr_gla_decode_step", 9)
+gdr_gla_decode_step_f32 = _gla_wrapper("gdr_gla_decode_step_f32", 9)
+
+
 def prefill(q, k, v, a, b, A_log, dt_bias, init_state=None, cu_seqlens=None, chunk=32,
-            form="chunked", out=None, final_state=None, stream=None):
+            form="chunked", out=None, final_state=None, stream=None, erase=True):
     """Prefill over q, k [B, T, Hk, dk], v [B, T, Hv, dv], a, b [B, T, Hv] (bf16 or fp32).
 
     ``form`` is "chunked" (UT transform) or "recurrent".  With ``cu_seqlens`` (int32,
     device, [N + 1]) the tokens are packed along T (B must be 1) into N sequences.
+    ``erase=False`` runs gated linear attention (the rule without its erase term).
     Returns (out [B, T, Hv, dv] fp32, final_state [Nseq, Hv, dk, dv] fp32).
     """
     import torch
@@ -213,17 +237,22 @@ def prefill(q, k, v, a, b, A_log, dt_bias, init_state=None, cu_seqlens=None, chu
     args = (q, k, v, a, b, A_log, dt_bias, init_state, out, final_state, cu_seqlens,
             nseq, B * T if cu_seqlens is not None else T, Hk, Hv, dk, dv)
     if form == "chunked":
-        (gdr_prefill_chunked_f32 if f32 else gdr_prefill_chunked)(*args, chunk, stream=stream)
+        fn = ((gdr_prefill_chunked_f32 if f32 else gdr_prefill_chunked) if erase else
+              (gdr_gla_prefill_chunked_f32 if f32 else gdr_gla_prefill_chunked))
+        fn(*args, chunk, stream=stream)
     elif form == "recurrent":
-        (gdr_prefill_recurrent_f32 if f32 else gdr_prefill_recurrent)(*args, stream=stream)
+        fn = ((gdr_prefill_recurrent_f32 if f32 else gdr_prefill_recurrent) if erase else
+              (gdr_gla_prefill_recurrent_f32 if f32 else gdr_gla_prefill_recurrent))
+        fn(*args, stream=stream)
     else:
         raise ValueError(f"unknown form {form!r}")
     return out, final_state
 
 
-def decode_step(q, k, v, a, b, A_log, dt_bias, state, out=None, stream=None):
+def decode_step(q, k, v, a, b, A_log, dt_bias, state, out=None, stream=None, erase=True):
     """One recurrent step: q, k [B, Hk, dk], v [B, Hv, dv], a, b [B, Hv]; ``state``
-    [B, Hv, dk, dv] fp32 is updated in place.  Returns out [B, Hv, dv] fp32."""
+    [B, Hv, dk, dv] fp32 is updated in place (``erase=False``: gated linear attention).
+    Returns out [B, Hv, dv] fp32."""
     import torch
 
     dtype = q.dtype
@@ -233,6 +262,8 @@ def decode_step(q, k, v, a, b, A_log, dt_bias, state, out=None, stream=None):
     Hv, dv = v.shape[1], v.shape[2]
     if out is None:
         out = torch.empty((B, Hv, dv), device=q.device, dtype=torch.float32)
-    fn = gdr_decode_step_f32 if dtype == torch.float32 else gdr_decode_step
+    f32 = dtype == torch.float32
+    fn = ((gdr_decode_step_f32 if f32 else gdr_decode_step) if erase else
+          (gdr_gla_decode_step_f32 if f32 else gdr_gla_decode_step))
     fn(q, k, v, a, b, A_log, dt_bias, state, out, B, Hk, Hv, dk, dv, stream=stream)
     return out

@@ -15,7 +15,9 @@
 //     Delta  = T (diag(beta) V - diag(beta exp(G)) K S)    = U - W S
 //     O      = diag(exp(G)) Q S + (Q K^T * M) Delta,       M[i,j] = exp(G_i - G_j), j <= i
 //     S'     = exp(G_C) S + (diag(exp(G_C - G)) K)^T Delta
-// All decay factors are exp of a non-positive number, so none overflows.
+// All decay factors are exp of a non-positive number, so none overflows.  With the erase
+// term off (gated linear attention; tessera PR #77 summary, "What landed": erase=False)
+// A = 0, so T = I and Delta = diag(beta) V.
 //
 // One CTA owns one (sequence, value head, 32-column slice of dv): the columns of S are
 // independent (delta_j, S[:, j] and o_j depend only on column j), so the slice's state
@@ -52,7 +54,8 @@ chunked_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
                     const Tin* __restrict__ a, const Tin* __restrict__ b,
                     const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                     const float* init_state, float* __restrict__ out, float* final_state,
-                    const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv, int dv) {
+                    const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv, int dv,
+                    int erase) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem<DK>& sm = *reinterpret_cast<SimtSmem<DK>*>(smem_raw);
     const int ntiles = dv / kDVT;
@@ -161,7 +164,7 @@ chunked_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
             for (int x = 0; x < 4; ++x) {
                 const int j = j0 + x;
                 const float dec = j <= i ? expf(Gi - sm.G[j]) : 0.f;
-                sm.A[i][j] = j < i ? bi * dec * kk[x] : 0.f;
+                sm.A[i][j] = (erase && j < i) ? bi * dec * kk[x] : 0.f;  // erase = 0: A = 0
                 sm.P[i][j] = dec * qk[x];
                 sm.KS[i][j] = ks[x];
                 sm.QS[i][j] = qs[x];
@@ -184,7 +187,7 @@ chunked_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
         } else {
             for (int e = tid - 32; e < kC * kDVT; e += kNT - 32) {
                 const int i = e / kDVT, c = e % kDVT;
-                sm.KS[i][c] = sm.beta[i] * (sm.V[i][c] - sm.eG[i] * sm.KS[i][c]);
+                sm.KS[i][c] = sm.beta[i] * (sm.V[i][c] - (erase ? sm.eG[i] * sm.KS[i][c] : 0.f));
             }
         }
         __syncthreads();
@@ -251,7 +254,7 @@ cudaError_t launch_typed(const FwdParams& p, cudaStream_t stream) {
     chunked_simt_kernel<DK, Tin><<<grid, kNT, smem, stream>>>(
         (const Tin*)p.q, (const Tin*)p.k, (const Tin*)p.v, (const Tin*)p.a, (const Tin*)p.b,
         p.A_log, p.dt_bias, p.init_state, p.out, p.final_state, p.cu_seqlens, p.T, p.Hk, p.Hv,
-        p.dv);
+        p.dv, p.erase);
     return cudaGetLastError();
 }
 

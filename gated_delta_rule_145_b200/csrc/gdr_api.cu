@@ -73,12 +73,18 @@ int prefill_recurrent(const FwdParams& p, cudaStream_t stream) {
 
 int decode_step(const void* q, const void* k, const void* v, const void* a, const void* b,
                 const float* A_log, const float* dt_bias, float* state, float* out, int B, int Hk,
-                int Hv, int dk, int dv, InType in, cudaStream_t stream) {
+                int Hv, int dk, int dv, InType in, cudaStream_t stream, int erase = 1) {
     if (!state) return GDR_ERR_NULL;
     // one token per sequence: the dense layout with T = 1, state updated in place
-    const FwdParams p = make_params(q, k, v, a, b, A_log, dt_bias, state, out, state, nullptr, B,
-                                    1, Hk, Hv, dk, dv, 0, in);
+    FwdParams p = make_params(q, k, v, a, b, A_log, dt_bias, state, out, state, nullptr, B, 1, Hk,
+                              Hv, dk, dv, 0, in);
+    p.erase = erase;
     return prefill_recurrent(p, stream);
+}
+
+FwdParams gla(FwdParams p) {
+    p.erase = 0;
+    return p;
 }
 
 }  // namespace
@@ -157,6 +163,67 @@ int gdr_decode_step_f32(const float* q, const float* k, const float* v, const fl
                         float* out, int B, int Hk, int Hv, int dk, int dv, gdr_stream_t stream) {
     return decode_step(q, k, v, a, b, A_log, dt_bias, state, out, B, Hk, Hv, dk, dv,
                        InType::F32, (cudaStream_t)stream);
+}
+
+// ---- erase=False: gated linear attention through the same kernels
+
+int gdr_gla_prefill_chunked(const void* q, const void* k, const void* v, const void* a,
+                            const void* b, const float* A_log, const float* dt_bias,
+                            const float* init_state, float* out, float* final_state,
+                            const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                            int dv, int chunk, gdr_stream_t stream) {
+    return prefill_chunked(gla(make_params(q, k, v, a, b, A_log, dt_bias, init_state, out,
+                                           final_state, cu_seqlens, B, T, Hk, Hv, dk, dv, chunk,
+                                           InType::BF16)),
+                           (cudaStream_t)stream);
+}
+
+int gdr_gla_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,
+                                const float* b, const float* A_log, const float* dt_bias,
+                                const float* init_state, float* out, float* final_state,
+                                const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                                int dv, int chunk, gdr_stream_t stream) {
+    return prefill_chunked(gla(make_params(q, k, v, a, b, A_log, dt_bias, init_state, out,
+                                           final_state, cu_seqlens, B, T, Hk, Hv, dk, dv, chunk,
+                                           InType::F32)),
+                           (cudaStream_t)stream);
+}
+
+int gdr_gla_prefill_recurrent(const void* q, const void* k, const void* v, const void* a,
+                              const void* b, const float* A_log, const float* dt_bias,
+                              const float* init_state, float* out, float* final_state,
+                              const int32_t* cu_seqlens, int B, int T, int Hk, int Hv, int dk,
+                              int dv, gdr_stream_t stream) {
+    return prefill_recurrent(gla(make_params(q, k, v, a, b, A_log, dt_bias, init_state, out,
+                                             final_state, cu_seqlens, B, T, Hk, Hv, dk, dv, 0,
+                                             InType::BF16)),
+                             (cudaStream_t)stream);
+}
+
+int gdr_gla_prefill_recurrent_f32(const float* q, const float* k, const float* v, const float* a,
+                                  const float* b, const float* A_log, const float* dt_bias,
+                                  const float* init_state, float* out, float* final_state,
+                                  const int32_t* cu_seqlens, int B, int T, int Hk, int Hv,
+                                  int dk, int dv, gdr_stream_t stream) {
+    return prefill_recurrent(gla(make_params(q, k, v, a, b, A_log, dt_bias, init_state, out,
+                                             final_state, cu_seqlens, B, T, Hk, Hv, dk, dv, 0,
+                                             InType::F32)),
+                             (cudaStream_t)stream);
+}
+
+int gdr_gla_decode_step(const void* q, const void* k, const void* v, const void* a,
+                        const void* b, const float* A_log, const float* dt_bias, float* state,
+                        float* out, int B, int Hk, int Hv, int dk, int dv, gdr_stream_t stream) {
+    return decode_step(q, k, v, a, b, A_log, dt_bias, state, out, B, Hk, Hv, dk, dv,
+                       InType::BF16, (cudaStream_t)stream, 0);
+}
+
+int gdr_gla_decode_step_f32(const float* q, const float* k, const float* v, const float* a,
+                            const float* b, const float* A_log, const float* dt_bias,
+                            float* state, float* out, int B, int Hk, int Hv, int dk, int dv,
+                            gdr_stream_t stream) {
+    return decode_step(q, k, v, a, b, A_log, dt_bias, state, out, B, Hk, Hv, dk, dv,
+                       InType::F32, (cudaStream_t)stream, 0);
 }
 
 int gdr_device_status(gdr_stream_t stream) {

@@ -18,6 +18,9 @@ struct FwdParams {
     const int32_t* cu_seqlens;      // [nseq + 1] or nullptr (dense: nseq sequences of T)
     int nseq, T, Hk, Hv, dk, dv, chunk;
     InType in;
+    // 1: the gated delta rule; 0: its erase=False special case, gated linear attention
+    // (delta = beta v, no k^T S term)
+    int erase = 1;
 };
 
 // Sequential recurrence (decode step and recurrent prefill); recurrent.cu.

@@ -23,6 +23,9 @@
 // Delta_{c+1} follows from Delta_c through one 32-deep product; the state enters only
 // through Y_{c+1}, which needs S_c, a chunk earlier.
 //
+// Without the erase term (gated linear attention, the erase=False case of tessera PR #77
+// summary, "What landed") A = 0 and Wt = M = 0: T = I, Delta = diag(beta) V.
+//
 // Precision.  Every tensor-core product has a raw bf16 input (exact) on one side or splits
 // an fp32 operand into bf16 hi + lo (about 16 significant bits); derived x derived
 // products take hi*hi + hi*lo + lo*hi.  Accumulation is fp32.  Decay factors are exp of
@@ -179,7 +182,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                    const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                    const int32_t* __restrict__ cu_seqlens, int T, int nseq, int Hk, int Hv,
-                   uint8_t* __restrict__ ws) {
+                   int erase, uint8_t* __restrict__ ws) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     PrepSmem& sm = *reinterpret_cast<PrepSmem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -311,7 +314,9 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int i = tid;
         const float rk = inv_norm_fast(sm.f.u.g.KK[i][i]);
         sm.rk[i] = rk;
-        sm.w[i] = sm.beta[i] * sm.eG[i] * rk;
+        // erase = 0 (gated linear attention): w = 0 and A = 0 below, so T = I, Wt = M = 0
+        // and the state-passing kernel's W terms vanish
+        sm.w[i] = erase ? sm.beta[i] * sm.eG[i] * rk : 0.f;
         vec[rec::VEC_E + i] = sm.eG[i] * sm.rq[i];
         vec[rec::VEC_D + i] = __expf(sm.G[C - 1] - sm.G[i]) * rk;
         if (i == 0) vec[rec::VEC_GAMMA] = __expf(sm.G[C - 1]);
@@ -331,7 +336,7 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int q = 0; q < 8; ++q) {
             const int j = j0 + q;
             const float dec = __expf(Gi - sm.G[j]) * sm.rk[j];  // used only where j <= i
-            am[q] = j < i ? fa * sm.f.u.g.KK[i][j] * dec : 0.f;
+            am[q] = (erase && j < i) ? fa * sm.f.u.g.KK[i][j] * dec : 0.f;
             pm[q] = j <= i ? fp * sm.f.u.g.QK[i][j] * dec : 0.f;
             r3[q] = wi * sm.f.u.g.KR[i][j] * sm.Dp[j];
         }
@@ -1038,7 +1043,7 @@ cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stre
     if (e != cudaSuccess) return e;
     intra_chunk_kernel<<<(unsigned)(nrec * p.Hv), PREP_THREADS, sizeof(PrepSmem), stream>>>(
         mq, mk, (const __nv_bfloat16*)p.a, (const __nv_bfloat16*)p.b, p.A_log, p.dt_bias,
-        p.cu_seqlens, p.T, p.nseq, p.Hk, p.Hv, (uint8_t*)ws);
+        p.cu_seqlens, p.T, p.nseq, p.Hk, p.Hv, p.erase, (uint8_t*)ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     state_pass_kernel<<<(unsigned)(p.nseq * p.Hv * NTILES), SP_THREADS, sizeof(SpSmem), stream>>>(

@@ -15,7 +15,8 @@
 //     delta = beta (v - gamma u)
 //     o     = gamma p + (q . k) delta        ( = q^T S_new )
 //     S_new = gamma S_old + k delta^T
-// so S is touched once per step.  Every warp normalises q and k itself (warp reductions,
+// so S is touched once per step.  Without the erase term (erase = 0: gated linear
+// attention, the erase=False case of tessera PR #77 summary, "What landed") delta = beta v.  Every warp normalises q and k itself (warp reductions,
 // no block barrier); the column sums over row groups cross warps through a double-
 // buffered shared array, one block barrier per token.
 #include "gdr_common.cuh"
@@ -68,7 +69,7 @@ recurrent_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
                  const Tin* __restrict__ a, const Tin* __restrict__ b,
                  const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                  const float* init_state, float* __restrict__ out, float* final_state,
-                 const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv) {
+                 const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv, int erase) {
     using Sh = RecShape<DK, DV, Tin>;
     constexpr int COLS = Sh::COLS, CG = Sh::CG, RG = Sh::RG, RPT = Sh::RPT, EPL = Sh::EPL;
     constexpr int NSLICE = DV / COLS;
@@ -156,10 +157,11 @@ recurrent_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             p.x += y.x; p.y += y.y; p.z += y.z; p.w += y.w;
         }
         float4 d;
-        d.x = beta * (vv.x - gam * u.x);
-        d.y = beta * (vv.y - gam * u.y);
-        d.z = beta * (vv.z - gam * u.z);
-        d.w = beta * (vv.w - gam * u.w);
+        const float ge = erase ? gam : 0.f;  // erase = 0: gated linear attention, delta = beta v
+        d.x = beta * (vv.x - ge * u.x);
+        d.y = beta * (vv.y - ge * u.y);
+        d.z = beta * (vv.z - ge * u.z);
+        d.w = beta * (vv.w - ge * u.w);
         if (rg == 0) {
             float4 o;
             o.x = gam * p.x + qk * d.x;
@@ -190,7 +192,8 @@ cudaError_t launch_typed(const FwdParams& p, cudaStream_t stream) {
     const dim3 grid((unsigned)(p.nseq * p.Hv * (D / Sh::COLS)));
     recurrent_kernel<D, D, Tin><<<grid, Sh::NT, 0, stream>>>(
         (const Tin*)p.q, (const Tin*)p.k, (const Tin*)p.v, (const Tin*)p.a, (const Tin*)p.b,
-        p.A_log, p.dt_bias, p.init_state, p.out, p.final_state, p.cu_seqlens, p.T, p.Hk, p.Hv);
+        p.A_log, p.dt_bias, p.init_state, p.out, p.final_state, p.cu_seqlens, p.T, p.Hk, p.Hv,
+        p.erase);
     return cudaGetLastError();
 }
 

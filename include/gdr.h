@@ -171,6 +171,45 @@ GDR_API int gdr_prefill_recurrent_f32(const float* q, const float* k, const floa
                               int dv, gdr_stream_t stream);
 
 /*
+ * erase=False: gated linear attention.  The pages treat the rule without its erase term
+ * as gated linear attention (tessera PR #77 summary, "The core finding (L0)" and "What
+ * landed": erase=False); these calls run that special case through the same kernels:
+ *     S <- S * exp(g_t);  delta <- v_t * beta_t;  S <- S + k_t (outer) delta;  o_t <- q_t^T S
+ * (q, k normalised and q scaled exactly as above).  Arguments, layouts, dispatch and
+ * status codes are those of the call without the "_gla" part of the name.
+ */
+GDR_API int gdr_gla_prefill_chunked(const void* q, const void* k, const void* v, const void* a,
+                                    const void* b, const float* A_log, const float* dt_bias,
+                                    const float* init_state, float* out, float* final_state,
+                                    const int32_t* cu_seqlens, int B, int T, int Hk, int Hv,
+                                    int dk, int dv, int chunk, gdr_stream_t stream);
+GDR_API int gdr_gla_prefill_chunked_f32(const float* q, const float* k, const float* v,
+                                        const float* a, const float* b, const float* A_log,
+                                        const float* dt_bias, const float* init_state,
+                                        float* out, float* final_state,
+                                        const int32_t* cu_seqlens, int B, int T, int Hk, int Hv,
+                                        int dk, int dv, int chunk, gdr_stream_t stream);
+GDR_API int gdr_gla_prefill_recurrent(const void* q, const void* k, const void* v,
+                                      const void* a, const void* b, const float* A_log,
+                                      const float* dt_bias, const float* init_state, float* out,
+                                      float* final_state, const int32_t* cu_seqlens, int B,
+                                      int T, int Hk, int Hv, int dk, int dv, gdr_stream_t stream);
+GDR_API int gdr_gla_prefill_recurrent_f32(const float* q, const float* k, const float* v,
+                                          const float* a, const float* b, const float* A_log,
+                                          const float* dt_bias, const float* init_state,
+                                          float* out, float* final_state,
+                                          const int32_t* cu_seqlens, int B, int T, int Hk,
+                                          int Hv, int dk, int dv, gdr_stream_t stream);
+GDR_API int gdr_gla_decode_step(const void* q, const void* k, const void* v, const void* a,
+                                const void* b, const float* A_log, const float* dt_bias,
+                                float* state, float* out, int B, int Hk, int Hv, int dk, int dv,
+                                gdr_stream_t stream);
+GDR_API int gdr_gla_decode_step_f32(const float* q, const float* k, const float* v,
+                                    const float* a, const float* b, const float* A_log,
+                                    const float* dt_bias, float* state, float* out, int B,
+                                    int Hk, int Hv, int dk, int dv, gdr_stream_t stream);
+
+/*
  * Device-side status of the kernels enqueued so far.  Synchronises `stream`, then returns
  * GDR_ERR_TIMEOUT if any tensor-core prefill kernel abandoned one of its bounded waits
  * (each wait on an mbarrier gives up after 2 s, records the event and lets the kernel

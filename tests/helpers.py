@@ -44,8 +44,9 @@ def to_device(inp, device="cuda"):
     return d
 
 
-def oracle_forward(inp, heads=None, nthreads=None):
-    """fp64 oracle on an Inputs bundle; optionally on a subset of value heads.
+def oracle_forward(inp, heads=None, nthreads=None, erase=True):
+    """fp64 oracle on an Inputs bundle; optionally on a subset of value heads; erase=False
+    gives gated linear attention.
 
     Returns (o, S) restricted to ``heads`` (value-head axis) when given.
     """
@@ -64,4 +65,4 @@ def oracle_forward(inp, heads=None, nthreads=None):
         A_log, dt_bias = A_log[heads], dt_bias[heads]
         S0 = None if S0 is None else S0[:, heads]
     return oracle.forward(q, k, v, a, b, A_log, dt_bias, S0, cu_seqlens=inp.cu_seqlens,
-                          nthreads=nthreads)
+                          nthreads=nthreads, erase=erase)
