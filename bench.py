@@ -285,6 +285,34 @@ def bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth):
     gla_steps = max(3, min(args.steps, 10))
     res.update(gla_ms=_timed(dist, dev, stream, sampler, gla, gla_steps), gla_steps=gla_steps,
                launches=res["launches"] + 2 * gla_steps)
+    # the steps around the rule at the same sizes: conv + SiLU over the q|k|v channels of
+    # every token, gated RMSNorm over every (token, head) row of the rule's output
+    C = 2 * P["Hk"] * P["dk"] + P["Hv"] * P["dv"]
+    g = torch.Generator(device=dev).manual_seed(7)
+    xc = torch.randn((P["B"], P["T"], C), device=dev, generator=g).to(torch.bfloat16)
+    yc = torch.empty_like(xc)
+    wc = torch.randn((C, 4), device=dev, generator=g) * 0.5
+    bc = torch.randn((C,), device=dev, generator=g) * 0.1
+    sc = torch.zeros((P["B"], C, 3), device=dev)
+    zr = torch.randn(out.shape, device=dev, generator=g).to(torch.bfloat16)
+    wr = torch.rand((P["dv"],), device=dev, generator=g) + 0.5
+    yr = torch.empty_like(out)
+    rows = P["B"] * P["T"] * P["Hv"]
+
+    def conv(_i):
+        gdr.gdr_short_conv_silu(xc, wc, bc, sc, sc, yc, P["B"], P["T"], C, stream=stream)
+
+    def norm(_i):
+        gdr.gdr_gated_rmsnorm(out, zr, wr, yr, rows, P["dv"], 1e-6, stream=stream)
+
+    io = {}
+    for name, fn, nbytes in (("conv_silu", conv, 2 * xc.numel() * 2 + sc.numel() * 8),
+                             ("gated_rmsnorm", norm, out.numel() * (4 + 2 + 4))):
+        for i in range(3):
+            fn(i)
+        ms = _timed(dist, dev, stream, sampler, fn, 10) / 10
+        io[name] = dict(ms=ms, bytes=nbytes)
+    res.update(mixer_io=io, launches=res["launches"] + 20)
     if args.no_e2e:
         return res
     # ---- end to end through the public API: pinned host inputs in, outputs back
@@ -409,6 +437,17 @@ def run_ours(args, dist):
                 "cpu_baseline": cpu,
             })
             result["gpu_launches"] += pre["launches"]
+            result["mixer_io"] = {
+                name: {"ms": round(v["ms"], 4), "alg_bytes": v["bytes"],
+                       "roofline": {"bound": "hbm",
+                                    "achieved": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1),
+                                    "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                    "frac": round(v["bytes"] / (v["ms"] / 1e3) / 1e9 /
+                                                  pk["hbm_gbs"], 4)}}
+                for name, v in pre["mixer_io"].items()}
+            result["mixer_io"]["workload"] = (
+                "conv_silu: x [1, 8192, 18432] bf16 (q|k|v channels, Hk=Hv=48, d=128), "
+                "4 taps, state in place; gated_rmsnorm: o [8192*48, 128] fp32, bf16 gate")
             gla_s = pre["gla_ms"] / pre["gla_steps"] / 1e3
             result["gla"] = {
                 "form": "erase=False (gated linear attention), same workload and kernels",

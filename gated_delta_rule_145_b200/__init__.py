@@ -58,6 +58,9 @@ _SIGS = {
     "gdr_gla_prefill_recurrent_f32": [_P] * 11 + [_I] * 6 + [_P],
     "gdr_gla_decode_step": [_P] * 9 + [_I] * 5 + [_P],
     "gdr_gla_decode_step_f32": [_P] * 9 + [_I] * 5 + [_P],
+    "gdr_short_conv_silu": [_P] * 6 + [_I] * 4 + [_P],
+    "gdr_gated_rmsnorm": [_P] * 4 + [ctypes.c_longlong, _I, ctypes.c_float, _P],
+    "gdr_gated_rmsnorm_f32": [_P] * 4 + [ctypes.c_longlong, _I, ctypes.c_float, _P],
 }
 
 
@@ -206,6 +209,32 @@ gdr_gla_prefill_recurrent = _gla_wrapper("gdr_gla_prefill_recurrent", 11)
 gdr_gla_prefill_recurrent_f32 = _gla_wrapper("gdr_gla_prefill_recurrent_f32", 11)
 gdr_gla_decode_step = _gla_wrapper("gdr_gla_decode_step", 9)
 gdr_gla_decode_step_f32 = _gla_wrapper("gdr_gla_decode_step_f32", 9)
+
+
+def gdr_short_conv_silu(x, weight, bias, conv_state_in, conv_state_out, y, B, T, C, width=4,
+                        stream=None, check=True):
+    """The four-tap causal convolution + SiLU before the rule (see include/gdr.h)."""
+    return _call("gdr_short_conv_silu", (x, weight, bias, conv_state_in, conv_state_out, y),
+                 (B, T, C, width), stream, check)
+
+
+def _norm_call(name, o, z, weight, y, rows, d, eps, stream, check):
+    fn = getattr(library(), name)
+    status = fn(_ptr(o), _ptr(z), _ptr(weight), _ptr(y), ctypes.c_longlong(int(rows)), int(d),
+                ctypes.c_float(eps), _stream(stream))
+    if check and status != GDR_OK:
+        raise GdrError(name, status)
+    return status
+
+
+def gdr_gated_rmsnorm(o, z, weight, y, rows, d, eps=1e-6, stream=None, check=True):
+    """The gated RMS normalisation after the rule, bf16 gate (see include/gdr.h)."""
+    return _norm_call("gdr_gated_rmsnorm", o, z, weight, y, rows, d, eps, stream, check)
+
+
+def gdr_gated_rmsnorm_f32(o, z, weight, y, rows, d, eps=1e-6, stream=None, check=True):
+    """The gated RMS normalisation after the rule, fp32 gate (see include/gdr.h)."""
+    return _norm_call("gdr_gated_rmsnorm_f32", o, z, weight, y, rows, d, eps, stream, check)
 
 
 def prefill(q, k, v, a, b, A_log, dt_bias, init_state=None, cu_seqlens=None, chunk=32,

@@ -226,6 +226,42 @@ int gdr_gla_decode_step_f32(const float* q, const float* k, const float* v, cons
                        InType::F32, (cudaStream_t)stream, 0);
 }
 
+// ---- the steps around the rule
+
+int gdr_short_conv_silu(const void* x, const float* weight, const float* bias,
+                        const float* conv_state_in, float* conv_state_out, void* y, int B, int T,
+                        int C, int width, gdr_stream_t stream) {
+    if (!weight || (T > 0 && (!x || !y))) return GDR_ERR_NULL;
+    if (B < 1 || T < 0 || C < 8 || C % 8 != 0) return GDR_ERR_SHAPE;
+    if (width != 4) return GDR_ERR_UNSUPPORTED;
+    if ((long long)B * C * ((long long)T + 64) > 0x3fffffffffffLL) return GDR_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(weight, 16) || !aligned(bias, 4) ||
+        !aligned(conv_state_in, 4) || !aligned(conv_state_out, 4))
+        return GDR_ERR_ALIGN;
+    return to_status(gdr::launch_short_conv_silu(x, weight, bias, conv_state_in, conv_state_out,
+                                                 y, B, T, C, (cudaStream_t)stream));
+}
+
+static int gated_rmsnorm(const float* o, const void* z, bool z_f32, const float* weight,
+                         float* y, long long rows, int d, float eps, cudaStream_t stream) {
+    if (!weight || (rows > 0 && (!o || !z || !y))) return GDR_ERR_NULL;
+    if (rows < 0 || !(eps >= 0.f)) return GDR_ERR_SHAPE;
+    if (d != 32 && d != 64 && d != 128) return GDR_ERR_UNSUPPORTED;
+    if (!aligned(o, 16) || !aligned(y, 16) || !aligned(z, z_f32 ? 16 : 8) || !aligned(weight, 4))
+        return GDR_ERR_ALIGN;
+    return to_status(gdr::launch_gated_rmsnorm(o, z, z_f32, weight, y, rows, d, eps, stream));
+}
+
+int gdr_gated_rmsnorm(const float* o, const void* z, const float* weight, float* y,
+                      long long rows, int d, float eps, gdr_stream_t stream) {
+    return gated_rmsnorm(o, z, false, weight, y, rows, d, eps, (cudaStream_t)stream);
+}
+
+int gdr_gated_rmsnorm_f32(const float* o, const float* z, const float* weight, float* y,
+                          long long rows, int d, float eps, gdr_stream_t stream) {
+    return gated_rmsnorm(o, z, true, weight, y, rows, d, eps, (cudaStream_t)stream);
+}
+
 int gdr_device_status(gdr_stream_t stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDR_ERR_CUDA;
     const int v = gdr::read_and_clear_tc_status();

@@ -43,6 +43,15 @@ cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stre
 // Returns the cached workspace memory of every device to the system; prefill_tc.cu.
 void workspace_release();
 
+// The steps around the rule (mixer_io.cu): the four-tap causal convolution + SiLU on bf16
+// channels (C a multiple of 8; state [B, C, 3] fp32, either pointer may be null, in place allowed),
+// and the gated RMS normalisation of fp32 rows of d values (z bf16 or fp32).
+cudaError_t launch_short_conv_silu(const void* x, const float* w, const float* bias,
+                                   const float* state_in, float* state_out, void* y, int B, int T,
+                                   int C, cudaStream_t stream);
+cudaError_t launch_gated_rmsnorm(const float* o, const void* z, bool z_f32, const float* weight,
+                                 float* y, long long rows, int d, float eps, cudaStream_t stream);
+
 // The fixed scratch area of the no-allocation prefill entry point: its size, and its
 // device address on the current device (looked up once per device); noalloc.cu.
 size_t noalloc_scratch_bytes();

@@ -1,0 +1,255 @@
+// mixer_io.cu -- the steps on either side of the gated delta rule in its mixer:
+//   short_conv_silu_kernel  before it: a short causal depthwise convolution over time
+//                           (four taps, kept as a ring buffer of the last three inputs
+//                           per channel) followed by SiLU, on the input projections;
+//   gated_rmsnorm_kernel    after it: RMS normalisation of each head's output over the
+//                           head dimension, times a per-channel weight, gated by SiLU of
+//                           a gate input.
+//
+// Sources: flashprove issue #32 "Qwen3.8-27B port" (the operator list: a four-tap short
+// convolution and sigmoid gates; the M2 design decisions: the short convolution and SiLU
+// before the rule, a gated RMS normalisation of its output after it); PLENA_Simulator
+// PR #113, "Mamba + KDA support: common state engine, hybrid DSE" (the short convolution
+// as a ring buffer: a shift, a per-channel weight stride, a bias; the newest tap alone
+// passes the input through).  Readings where the pages give no formula:
+//   conv   y_t[c] = bias[c] + sum_{i<4} w[c, i] x_{t-3+i}[c]  (w[c, 3]: newest tap); the
+//          three inputs before the call come from the state (oldest first), zeros
+//          without one; the state after the call holds the last three inputs.
+//   norm   y = o / sqrt(mean_d(o^2) + eps) * weight * SiLU(z), weight shared by heads.
+// Both are HBM-bound streaming passes: coalesced vector loads, streaming stores, no reuse.
+#include <algorithm>
+
+#include "gdr_common.cuh"
+#include "gdr_internal.h"
+
+namespace gdr {
+namespace {
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+
+// SiLU with the fast exponential and division (relative error ~1e-6): for bf16 outputs,
+// whose rounding step is 2^-8, this keeps the pass bound by memory, not by arithmetic.
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
+// ------------------------------------------------------------------------ conv + SiLU
+
+constexpr int kConvW = 4;       // taps
+constexpr int kConvSeg = 64;    // tokens per thread when the state is not updated in place
+constexpr int kConvThreads = 256;
+
+// Thread -> (sequence b, time segment, group of 8 channels).  Channels are the fastest
+// index, so a warp moves 512 contiguous bytes per token in 16-byte accesses.
+__device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+        f[2 * e] = v.x;
+        f[2 * e + 1] = v.y;
+    }
+}
+
+__global__ void __launch_bounds__(kConvThreads)
+short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ w,
+                       const float* __restrict__ bias, const float* state_in, float* state_out,
+                       __nv_bfloat16* __restrict__ y, int B, int T, int C, int seg) {
+    constexpr int G = 8;  // channels per thread
+    const int groups = C / G;
+    const int nseg = (T + seg - 1) / seg;
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long total = (long long)B * nseg * groups;
+    if (gid >= total) return;
+    const int cg = (int)(gid % groups);
+    const long long r = gid / groups;
+    const int s = (int)(r % nseg), b = (int)(r / nseg);
+    const int c = G * cg;
+    const int t0 = s * seg, t1 = min(T, t0 + seg);
+    float wt[G][kConvW], bs[G];
+#pragma unroll
+    for (int e = 0; e < G; ++e) {
+        const float4 v = *reinterpret_cast<const float4*>(w + (size_t)(c + e) * kConvW);
+        wt[e][0] = v.x; wt[e][1] = v.y; wt[e][2] = v.z; wt[e][3] = v.w;
+        bs[e] = bias ? bias[c + e] : 0.f;
+    }
+    // window: the three inputs before t0 (oldest first)
+    float h[kConvW - 1][G];
+#pragma unroll
+    for (int j = 0; j < kConvW - 1; ++j) {
+        const int t = t0 - (kConvW - 1) + j;
+        if (t >= 0) {
+            unpack8(*reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * C + c), h[j]);
+        } else {
+            // state[b][c][j'] holds the input at time j' - 3 of this call
+            const int jj = t + (kConvW - 1);
+#pragma unroll
+            for (int e = 0; e < G; ++e)
+                h[j][e] = state_in ? state_in[((size_t)b * C + c + e) * (kConvW - 1) + jj] : 0.f;
+        }
+    }
+    const __nv_bfloat16* xp = x + ((size_t)b * T + t0) * C + c;
+    __nv_bfloat16* yp = y + ((size_t)b * T + t0) * C + c;
+#pragma unroll 8
+    for (int t = t0; t < t1; ++t, xp += C, yp += C) {
+        float v[G];
+        unpack8(__ldcs(reinterpret_cast<const uint4*>(xp)), v);
+        uint32_t o[G / 2];
+#pragma unroll
+        for (int e = 0; e < G; e += 2) {
+            const float a0 = bs[e] + wt[e][0] * h[0][e] + wt[e][1] * h[1][e] + wt[e][2] * h[2][e] +
+                             wt[e][3] * v[e];
+            const float a1 = bs[e + 1] + wt[e + 1][0] * h[0][e + 1] + wt[e + 1][1] * h[1][e + 1] +
+                             wt[e + 1][2] * h[2][e + 1] + wt[e + 1][3] * v[e + 1];
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(silu_fast(a0), silu_fast(a1));
+            o[e / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        __stcs(reinterpret_cast<uint4*>(yp), make_uint4(o[0], o[1], o[2], o[3]));
+#pragma unroll
+        for (int e = 0; e < G; ++e) {
+            h[0][e] = h[1][e];
+            h[1][e] = h[2][e];
+            h[2][e] = v[e];
+        }
+    }
+    // The new state (the last three inputs) is written by the thread of segment 0, the one
+    // that read the old state, so the state may be updated in place whatever the number of
+    // segments: with T >= 3 it is read back from x, with T < 3 (one segment) it is the
+    // window after the loop.
+    if (state_out && s == 0) {
+#pragma unroll
+        for (int j = 0; j < kConvW - 1; ++j) {
+            if (T >= kConvW - 1)
+                unpack8(*reinterpret_cast<const uint4*>(
+                            x + ((size_t)b * T + T - (kConvW - 1) + j) * C + c),
+                        h[j]);
+#pragma unroll
+            for (int e = 0; e < G; ++e)
+                state_out[((size_t)b * C + c + e) * (kConvW - 1) + j] = h[j][e];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------- gated RMSNorm
+
+constexpr int kNormThreads = 256;
+
+template <typename Tz>
+__device__ __forceinline__ void load_z(const Tz* p, float (&z)[4], int n);
+
+template <>
+__device__ __forceinline__ void load_z(const float* p, float (&z)[4], int n) {
+    if (n == 4) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(p));
+        z[0] = v.x; z[1] = v.y; z[2] = v.z; z[3] = v.w;
+    } else {
+        for (int e = 0; e < n; ++e) z[e] = __ldcs(p + e);
+    }
+}
+
+template <>
+__device__ __forceinline__ void load_z(const __nv_bfloat16* p, float (&z)[4], int n) {
+    if (n == 4) {
+        const float4 v = load4(p);
+        z[0] = v.x; z[1] = v.y; z[2] = v.z; z[3] = v.w;
+    } else {
+        for (int e = 0; e < n; ++e) z[e] = __bfloat162float(p[e]);
+    }
+}
+
+// One warp per row of d = 32 * EPL values; grid-stride over rows.
+template <typename Tz, int EPL>
+__global__ void __launch_bounds__(kNormThreads)
+gated_rmsnorm_kernel(const float* __restrict__ o, const Tz* __restrict__ z,
+                     const float* __restrict__ weight, float* __restrict__ y, long long rows,
+                     float eps) {
+    constexpr int D = 32 * EPL;
+    const int lane = threadIdx.x % 32;
+    float wl[4];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) wl[e] = weight[EPL * lane + e];
+    const long long warps = (long long)gridDim.x * (kNormThreads / 32);
+    for (long long row = (long long)blockIdx.x * (kNormThreads / 32) + threadIdx.x / 32;
+         row < rows; row += warps) {
+        const float* op = o + row * D + EPL * lane;
+        float ov[4], zv[4];
+        if constexpr (EPL == 4) {
+            const float4 v = __ldcs(reinterpret_cast<const float4*>(op));
+            ov[0] = v.x; ov[1] = v.y; ov[2] = v.z; ov[3] = v.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) ov[e] = __ldcs(op + e);
+        }
+        load_z(z + row * D + EPL * lane, zv, EPL);
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) ss += ov[e] * ov[e];
+        ss = warp_sum(ss);
+        const float r = 1.0f / sqrtf(ss / (float)D + eps);
+        float out[4];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) out[e] = ov[e] * r * wl[e] * silu_f(zv[e]);
+        float* yp = y + row * D + EPL * lane;
+        if constexpr (EPL == 4) {
+            __stcs(reinterpret_cast<float4*>(yp), make_float4(out[0], out[1], out[2], out[3]));
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) __stcs(yp + e, out[e]);
+        }
+    }
+}
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+template <typename Tz>
+cudaError_t launch_norm_typed(const float* o, const Tz* z, const float* weight, float* y,
+                              long long rows, int d, float eps, cudaStream_t stream) {
+    // enough resident warps to cover HBM latency: 8 CTAs of 8 warps per SM, grid-stride
+    const long long need = (rows + kNormThreads / 32 - 1) / (kNormThreads / 32);
+    const unsigned grid = (unsigned)std::min<long long>(need, (long long)sm_count() * 8);
+    if (grid == 0) return cudaSuccess;
+    switch (d) {
+        case 32: gated_rmsnorm_kernel<Tz, 1><<<grid, kNormThreads, 0, stream>>>(o, z, weight, y, rows, eps); break;
+        case 64: gated_rmsnorm_kernel<Tz, 2><<<grid, kNormThreads, 0, stream>>>(o, z, weight, y, rows, eps); break;
+        case 128: gated_rmsnorm_kernel<Tz, 4><<<grid, kNormThreads, 0, stream>>>(o, z, weight, y, rows, eps); break;
+        default: return cudaErrorNotSupported;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_short_conv_silu(const void* x, const float* w, const float* bias,
+                                   const float* state_in, float* state_out, void* y, int B, int T,
+                                   int C, cudaStream_t stream) {
+    if (T == 0) {
+        // nothing to convolve: the state passes through
+        if (state_out && state_in && state_out != state_in)
+            return cudaMemcpyAsync(state_out, state_in, sizeof(float) * B * C * (kConvW - 1),
+                                   cudaMemcpyDeviceToDevice, stream);
+        if (state_out && !state_in)
+            return cudaMemsetAsync(state_out, 0, sizeof(float) * B * C * (kConvW - 1), stream);
+        return cudaSuccess;
+    }
+    const int seg = kConvSeg;
+    const long long total = (long long)B * ((T + seg - 1) / seg) * (C / 8);
+    const unsigned grid = (unsigned)((total + kConvThreads - 1) / kConvThreads);
+    short_conv_silu_kernel<<<grid, kConvThreads, 0, stream>>>(
+        (const __nv_bfloat16*)x, w, bias, state_in, state_out, (__nv_bfloat16*)y, B, T, C, seg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gated_rmsnorm(const float* o, const void* z, bool z_f32, const float* weight,
+                                 float* y, long long rows, int d, float eps, cudaStream_t stream) {
+    return z_f32 ? launch_norm_typed(o, (const float*)z, weight, y, rows, d, eps, stream)
+                 : launch_norm_typed(o, (const __nv_bfloat16*)z, weight, y, rows, d, eps, stream);
+}
+
+}  // namespace gdr

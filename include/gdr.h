@@ -210,6 +210,40 @@ GDR_API int gdr_gla_decode_step_f32(const float* q, const float* k, const float*
                                     int Hk, int Hv, int dk, int dv, gdr_stream_t stream);
 
 /*
+ * The steps on either side of the rule in its mixer.  Sources: flashprove issue #32
+ * "Qwen3.8-27B port" (its operator list names a four-tap short convolution and sigmoid
+ * gates; its M2 design decisions place the short convolution and SiLU before the rule
+ * and a gated RMS normalisation of the rule's output after it); PLENA_Simulator PR #113,
+ * "Mamba + KDA support: common state engine, hybrid DSE" (the short convolution kept as
+ * a ring buffer: a shift, a per-channel weight stride, a bias).  The pages give no
+ * formulas; the readings below are this library's.
+ *
+ * gdr_short_conv_silu: per channel c of x [B, T, C] bf16 (the input projections, e.g.
+ * the q, k and v channels side by side), y_t[c] = SiLU(bias[c] + sum_{i<4} weight[c*4+i]
+ * x_{t-3+i}[c]) written as bf16 [B, T, C] (round to nearest even); weight[c*4+3] is the
+ * newest tap.  The three inputs before the call come from conv_state_in [B, C, 3] fp32
+ * (oldest first; NULL = zeros); conv_state_out [B, C, 3] receives the last three inputs
+ * (NULL to skip) and may be the same buffer as conv_state_in.  bias may be NULL.  C must
+ * be a multiple of 8; width must be 4; x, y and weight 16-byte aligned, the other
+ * pointers 4-byte aligned.  A decode step is a call with T = 1.
+ */
+GDR_API int gdr_short_conv_silu(const void* x, const float* weight, const float* bias,
+                                const float* conv_state_in, float* conv_state_out, void* y,
+                                int B, int T, int C, int width, gdr_stream_t stream);
+
+/*
+ * gdr_gated_rmsnorm: for each of `rows` rows of d values (one (token, head) of the rule's
+ * fp32 output o), y = o / sqrt(mean(o^2) + eps) * weight * SiLU(z), weight [d] fp32
+ * shared by all rows, z bf16 (the _f32 variant: fp32) with o's layout; y fp32.
+ * d in {32, 64, 128}; eps >= 0 (1e-6 is the value used with the rule); o, y (and an fp32
+ * z) 16-byte aligned, a bf16 z 8-byte aligned.
+ */
+GDR_API int gdr_gated_rmsnorm(const float* o, const void* z, const float* weight, float* y,
+                              long long rows, int d, float eps, gdr_stream_t stream);
+GDR_API int gdr_gated_rmsnorm_f32(const float* o, const float* z, const float* weight, float* y,
+                                  long long rows, int d, float eps, gdr_stream_t stream);
+
+/*
  * Device-side status of the kernels enqueued so far.  Synchronises `stream`, then returns
  * GDR_ERR_TIMEOUT if any tensor-core prefill kernel abandoned one of its bounded waits
  * (each wait on an mbarrier gives up after 2 s, records the event and lets the kernel

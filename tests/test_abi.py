@@ -99,3 +99,23 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         gdr.prefill(x, x, x, torch.zeros(1, 4, 1), torch.zeros(1, 4, 1), torch.zeros(1),
                     torch.zeros(1))
+
+
+def test_mixer_io_argument_errors():
+    conv = lambda **kw: gdr.gdr_short_conv_silu(**{**dict(
+        x=A, weight=A + 256, bias=None, conv_state_in=None, conv_state_out=None, y=A + 512,
+        B=1, T=16, C=64, width=4), **kw}, stream=0, check=False)
+    assert conv(x=None) == gdr.GDR_ERR_NULL
+    assert conv(C=60) == gdr.GDR_ERR_SHAPE
+    assert conv(B=0) == gdr.GDR_ERR_SHAPE
+    assert conv(width=3) == gdr.GDR_ERR_UNSUPPORTED
+    assert conv(y=A + 8) == gdr.GDR_ERR_ALIGN
+    norm = lambda fn=gdr.gdr_gated_rmsnorm, **kw: fn(**{**dict(
+        o=A, z=A + 256, weight=A + 512, y=A + 768, rows=10, d=128, eps=1e-6), **kw},
+        stream=0, check=False)
+    assert norm(o=None) == gdr.GDR_ERR_NULL
+    assert norm(d=96) == gdr.GDR_ERR_UNSUPPORTED
+    assert norm(rows=-1) == gdr.GDR_ERR_SHAPE
+    assert norm(eps=-1.0) == gdr.GDR_ERR_SHAPE
+    assert norm(y=A + 8) == gdr.GDR_ERR_ALIGN
+    assert norm(gdr.gdr_gated_rmsnorm_f32, z=A + 8) == gdr.GDR_ERR_ALIGN
