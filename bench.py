@@ -333,7 +333,7 @@ def bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth):
     for i in range(min(args.warmup, 3)):
         e2e(i)
     e2e_ms = _timed(dist, dev, stream, sampler, e2e, e2e_steps)
-    res.update(e2e_steps=e2e_steps, e2e_ms=e2e_ms, launches=2 * (args.steps + e2e_steps),
+    res.update(e2e_steps=e2e_steps, e2e_ms=e2e_ms, launches=res["launches"] + 2 * e2e_steps,
                h2d=sum(t.numel() * t.element_size() for t in host.values()),
                d2h=out_h.numel() * 4 + fin_h.numel() * 4)
     return res

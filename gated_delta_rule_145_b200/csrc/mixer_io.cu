@@ -36,6 +36,7 @@ __device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f 
 constexpr int kConvW = 4;       // taps
 constexpr int kConvSeg = 64;    // tokens per thread when the state is not updated in place
 constexpr int kConvThreads = 256;
+constexpr int kConvBatch = 8;   // tokens whose loads a thread issues together
 
 // Thread -> (sequence b, time segment, group of 8 channels).  Channels are the fastest
 // index, so a warp moves 512 contiguous bytes per token in 16-byte accesses.
@@ -88,10 +89,10 @@ short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restr
     }
     const __nv_bfloat16* xp = x + ((size_t)b * T + t0) * C + c;
     __nv_bfloat16* yp = y + ((size_t)b * T + t0) * C + c;
-#pragma unroll 8
-    for (int t = t0; t < t1; ++t, xp += C, yp += C) {
+    // one token: SiLU(conv) of input v against the window h, then shift v into the window
+    auto step = [&](const uint4 raw, __nv_bfloat16* dst) {
         float v[G];
-        unpack8(__ldcs(reinterpret_cast<const uint4*>(xp)), v);
+        unpack8(raw, v);
         uint32_t o[G / 2];
 #pragma unroll
         for (int e = 0; e < G; e += 2) {
@@ -102,14 +103,28 @@ short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restr
             const __nv_bfloat162 pr = __floats2bfloat162_rn(silu_fast(a0), silu_fast(a1));
             o[e / 2] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        __stcs(reinterpret_cast<uint4*>(yp), make_uint4(o[0], o[1], o[2], o[3]));
+        __stcs(reinterpret_cast<uint4*>(dst), make_uint4(o[0], o[1], o[2], o[3]));
 #pragma unroll
         for (int e = 0; e < G; ++e) {
             h[0][e] = h[1][e];
             h[1][e] = h[2][e];
             h[2][e] = v[e];
         }
+    };
+    // Groups of kConvBatch tokens: all of a group's loads are issued before its first use,
+    // so each thread keeps that many 16-byte reads in flight.
+    int t = t0;
+    for (; t + kConvBatch <= t1; t += kConvBatch, xp += (size_t)kConvBatch * C,
+                                 yp += (size_t)kConvBatch * C) {
+        uint4 raw[kConvBatch];
+#pragma unroll
+        for (int u = 0; u < kConvBatch; ++u)
+            raw[u] = __ldcs(reinterpret_cast<const uint4*>(xp + (size_t)u * C));
+#pragma unroll
+        for (int u = 0; u < kConvBatch; ++u) step(raw[u], yp + (size_t)u * C);
     }
+#pragma unroll 1
+    for (; t < t1; ++t, xp += C, yp += C) step(__ldcs(reinterpret_cast<const uint4*>(xp)), yp);
     // The new state (the last three inputs) is written by the thread of segment 0, the one
     // that read the old state, so the state may be updated in place whatever the number of
     // segments: with T >= 3 it is read back from x, with T < 3 (one segment) it is the
