@@ -2,11 +2,11 @@
 // cores, in fp32.  It serves the fp32 inputs and the head sizes the tensor-core kernel
 // does not take.
 //
-// Sources: Mila "GatedDeltaRule.ixx File Reference", Detailed Description ("prefill runs
-// the chunked (UT-transform) form, which regroups the identical arithmetic into one
-// triangular solve per 32 steps"); tessera PR #77 summary, "What landed"
-// (gated_delta_rule_chunked: "the only non-GEMM step is the (I+A)^-1 forward
-// substitution").
+// Sources: Mila "GatedDeltaRule.ixx File Reference", Detailed Description (prefill
+// uses the chunked UT-transform form: the same arithmetic as the recurrence, grouped so
+// that each 32-token chunk needs a single triangular solve); tessera PR #77 summary,
+// "What landed" (gated_delta_rule_chunked: apart from the forward substitution for
+// (I + A)^-1, every step is a matrix product).
 //
 // Chunk algebra (derived from the step by substituting it into itself).  In a chunk of
 // C tokens with start state S, G_i = sum_{j<=i} g_j, normalised rows k_i, q_i:

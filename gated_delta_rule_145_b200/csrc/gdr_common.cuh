@@ -2,7 +2,7 @@
 //
 // Gate and normalisation formulas: Mila "GatedDeltaRule.ixx File Reference", Detailed
 // Description (beta = sigmoid(b), g = -exp(A_log) * softplus(a + dt_bias); q and k
-// L2-normalised, q scaled by 1/sqrt(head_key_dim)).
+// normalised to unit L2 norm, q then multiplied by dk^-1/2).
 #pragma once
 
 #include <cuda_bf16.h>

@@ -3,7 +3,7 @@
 //
 // Source: Mila "GatedDeltaRule.ixx File Reference", Detailed Description: per value head
 // a state S[dk][dv]; each step S <- S exp(g); delta <- (v - k^T S) beta;
-// S <- S + k (outer) delta; o <- q^T S ("Decode runs the sequential recurrence above").
+// S <- S + k (outer) delta; o <- q^T S.  Decode uses this sequential form.
 //
 // One CTA owns one (sequence, value head, slice of COLS state columns) for the whole call:
 // the columns of S are independent (delta_j, S[:, j] and o_j depend only on column j), so

@@ -5,9 +5,9 @@ callers.  It draws random numbers and rounds them to the storage type; it holds 
 of the method's arithmetic.
 
 Workload shapes follow the pages: a 128 x 128 state per head (flashprove issue #32
-"Qwen3.8-27B port", M1: "one Gated DeltaNet head at real 128x128 state"), 48 value
-heads ("the 48-head cost is extrapolated", same issue, M2) and 32-step chunks (Mila
-"GatedDeltaRule.ixx File Reference": "one triangular solve per 32 steps").  No
+"Qwen3.8-27B port", milestone M1: a single head with the full-size state), 48 value
+heads (same issue, M2: the cost of all 48 heads is estimated from one) and 32-step
+chunks (Mila "GatedDeltaRule.ixx File Reference": a triangular solve per 32 tokens).  No
 dataset or trained weight is involved; every tensor is drawn here.
 
 Recipe (numpy PCG64, ``default_rng(seed)``), drawn in this order:

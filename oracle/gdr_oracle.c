@@ -54,8 +54,8 @@ void oracle_gating(double a, double b, double A_log, double dt_bias, double* g, 
     *beta = sigmoid(b);
 }
 
-/* L2 normalisation over n elements, times `scale` ("GatedDeltaRule.ixx":
- * q and k L2-normalized, q scaled by 1/sqrt(head_key_dim)). */
+/* L2 normalisation over n elements, times `scale` ("GatedDeltaRule.ixx": q and k are
+ * brought to unit L2 norm, and q is then multiplied by dk^-1/2). */
 static void l2_normalise(const float* x, int n, double scale, double* out) {
     double ss = 0.0;
     for (int i = 0; i < n; ++i) ss += (double)x[i] * (double)x[i];

@@ -20,13 +20,13 @@ Sources (page title and section):
   * Mila "GatedDeltaRule.ixx File Reference", Detailed Description -- the step
     S <- S exp(g); delta <- (v - k^T S) beta; S <- S + k (x) delta; o <- q^T S,
     q/k L2 normalisation, q scaled by 1/sqrt(dk), beta = sigmoid(b),
-    g = -exp(A_log) softplus(a + dt_bias); "TWO FORMS, ONE DEFINITION": the chunked
-    form regroups the same arithmetic into one triangular solve per 32 steps.
+    g = -exp(A_log) softplus(a + dt_bias); the same section states that the chunked
+    form is the same arithmetic regrouped, with one triangular solve per 32 tokens.
   * tessera PR #77 "Track L -- genuine gated delta rule + Mamba2 SSM", summary
     ("The core finding (L0)", "What landed"): the (I - beta k k^T) erase term, the
     independent brute-force check, erase=False being gated linear attention, and
-    the chunked UT form whose only non-GEMM step is the (I + A)^-1 forward
-    substitution.
+    the chunked UT form, in which everything except the forward substitution for
+    (I + A)^-1 is a matrix product.
 
 Every function here is pinned by ``tests/test_oracle.py``; no function is
 "parity unpinned".
