@@ -24,6 +24,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -375,6 +376,76 @@ def bench_decode(args, dist, dev, stream, sampler, gdr, synth):
                 kernel_ms=statistics.mean(s.elapsed_time(e) for evs in ev for s, e in evs))
 
 
+def bench_cp(args, dist, dev, stream, sampler, gdr):
+    """Context-parallel prefill (segment maps, composition, prefill from each segment's
+    start state), two measurements on this GPU:
+      one_gpu   -- long context with few heads (B=1, T=65536, Hk=Hv=8): the plain prefill
+                   keeps 24 CTAs busy for 2048 chunk steps; gdr_prefill_chunked_cp runs 6
+                   segments side by side;
+      per_rank  -- one rank's share of an 8-GPU split of B=1, T=65536, Hk=Hv=48: its 8192
+                   tokens' maps, the composition of 8 maps and its prefill (the all-gather
+                   of 8 x 2 x 3.1 MB over NVLink is not included)."""
+    import torch
+
+    g = torch.Generator(device=dev).manual_seed(11 + dist.rank)
+
+    def draw(T, H):
+        r = lambda *shape: torch.randn(shape, device=dev, generator=g).to(torch.bfloat16)
+        A_log = torch.rand((H,), device=dev, generator=g) * math.log(16.0)
+        dt = torch.exp(torch.rand((H,), device=dev, generator=g) *
+                       (math.log(1e-1) - math.log(1e-3)) + math.log(1e-3))
+        return dict(q=r(1, T, H, 128), k=r(1, T, H, 128), v=r(1, T, H, 128), a=r(1, T, H),
+                    b=r(1, T, H), A_log=A_log, dt_bias=torch.log(torch.expm1(dt)))
+
+    def timed(fn, n=3):
+        fn(0)
+        return _timed(dist, dev, stream, sampler, fn, n) / n
+
+    res = {}
+    T, H, nseg = 65536, 8, 6
+    x = draw(T, H)
+    out = torch.empty((1, T, H, 128), device=dev)
+    fin = torch.empty((1, H, 128, 128), device=dev)
+    args_in = (x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"])
+    plain = timed(lambda _i: gdr.gdr_prefill_chunked(*args_in, None, out, fin, None, 1, T, H, H,
+                                                     128, 128, 32, stream=stream))
+    cp = timed(lambda _i: gdr.gdr_prefill_chunked_cp(*args_in, None, out, fin, T, H, H, 128, 128,
+                                                     32, nseg, stream=stream))
+    res["one_gpu"] = dict(workload=f"B=1 T={T} Hk=Hv={H} d=128 bf16, {nseg} segments",
+                          plain_ms=round(plain, 4), cp_ms=round(cp, 4),
+                          cp_tokens_per_s=round(T / (cp / 1e3), 1),
+                          alg_bytes=prefill_alg_bytes(1, T, H, H, 128, 128))
+    del x, out
+    G, Tr, H = 8, 8192, 48
+    x = draw(Tr, H)
+    args_in = (x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"])
+    out = torch.empty((1, Tr, H, 128), device=dev)
+    phi = torch.empty((1, H, 128, 128), device=dev)
+    nmap = torch.empty_like(phi)
+    phi_all = torch.empty((G, H, 128, 128), device=dev)
+    nmap_all = torch.empty_like(phi_all)
+    seg = torch.empty_like(phi_all)
+
+    def rank_work(_i):
+        gdr.gdr_prefill_segment_maps(*args_in, phi, nmap, None, 1, Tr, H, H, 128, 128, 32,
+                                     stream=stream)
+        phi_all.copy_(phi.expand(G, -1, -1, -1))  # stands in for the all-gather
+        nmap_all.copy_(nmap.expand(G, -1, -1, -1))
+        gdr.gdr_segment_combine(phi_all, nmap_all, None, seg, fin.new_empty((1, H, 128, 128)),
+                                G, H, 128, 128, stream=stream)
+        gdr.gdr_prefill_chunked(*args_in, seg[3:4], out, None, None, 1, Tr, H, H, 128, 128, 32,
+                                stream=stream)
+
+    per = timed(rank_work)
+    res["per_rank"] = dict(workload=f"rank 3 of {G}: B=1 T={G * Tr} Hk=Hv={H} d=128 bf16, "
+                                    f"{Tr} tokens per rank",
+                           ms=round(per, 4),
+                           implied_tokens_per_s=round(G * Tr / (per / 1e3), 1),
+                           note="one rank's measured work; the exchange is not included")
+    res["launches"] = 4 * 2 + 4 * 8 + 4 * 7  # plain, cp, rank work (1 warm-up + 3 each)
+    return res
+
+
 def run_ours(args, dist):
     import torch
 
@@ -396,6 +467,9 @@ def run_ours(args, dist):
         pre = bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth)
     if args.only in (None, "decode"):
         dec = bench_decode(args, dist, dev, stream, sampler, gdr, synth)
+    cpx = None
+    if args.only in (None, "cp"):
+        cpx = bench_cp(args, dist, dev, stream, sampler, gdr)
     sampler.stop()
     clocks = sampler.summary()
 
@@ -477,6 +551,13 @@ def run_ours(args, dist):
                              "alg_bytes_per_launch": dalg,
                              "kernel_ms": round(dec["kernel_ms"], 5)}}
             result["gpu_launches"] += dec["steps"]
+        if cpx is not None:
+            result["gpu_launches"] += cpx.pop("launches")
+            one = cpx["one_gpu"]
+            ach = one["alg_bytes"] / (one["cp_ms"] / 1e3) / 1e9
+            one["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4)}
+            result["context_parallel"] = cpx
     dist.close()
     return result
 
@@ -556,7 +637,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=128,
                     help="tokens per reference-arm step (all 48 heads)")
-    ap.add_argument("--only", choices=("prefill", "decode"), default=None,
+    ap.add_argument("--only", choices=("prefill", "decode", "cp"), default=None,
                     help="time one path only (profiling runs; not the contract line)")
     ap.add_argument("--T", type=int, default=0, help="prefill length override (profiling)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")

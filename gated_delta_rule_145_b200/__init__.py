@@ -61,6 +61,9 @@ _SIGS = {
     "gdr_short_conv_silu": [_P] * 6 + [_I] * 4 + [_P],
     "gdr_gated_rmsnorm": [_P] * 4 + [ctypes.c_longlong, _I, ctypes.c_float, _P],
     "gdr_gated_rmsnorm_f32": [_P] * 4 + [ctypes.c_longlong, _I, ctypes.c_float, _P],
+    "gdr_prefill_segment_maps": [_P] * 10 + [_I] * 7 + [_P],
+    "gdr_segment_combine": [_P] * 5 + [_I] * 4 + [_P],
+    "gdr_prefill_chunked_cp": [_P] * 10 + [_I] * 7 + [_P],
 }
 
 
@@ -140,6 +143,29 @@ def gdr_prefill_chunked_noalloc(q, k, v, a, b, A_log, dt_bias, init_state, out, 
     return _call("gdr_prefill_chunked_noalloc",
                  (q, k, v, a, b, A_log, dt_bias, init_state, out, final_state, cu_seqlens),
                  (B, T, Hk, Hv, dk, dv, chunk), stream, check)
+
+
+def gdr_prefill_segment_maps(q, k, v, a, b, A_log, dt_bias, phi, nmap, cu_seqlens, B, T, Hk,
+                             Hv, dk, dv, chunk, stream=None, check=True):
+    """Per-segment state maps S_end = phi S_start + nmap of B segments (include/gdr.h)."""
+    return _call("gdr_prefill_segment_maps",
+                 (q, k, v, a, b, A_log, dt_bias, phi, nmap, cu_seqlens),
+                 (B, T, Hk, Hv, dk, dv, chunk), stream, check)
+
+
+def gdr_segment_combine(phi, nmap, init_state, seg_init, final_state, G, Hv, dk, dv,
+                        stream=None, check=True):
+    """Composes G segment maps in order into start states and the final state."""
+    return _call("gdr_segment_combine", (phi, nmap, init_state, seg_init, final_state),
+                 (G, Hv, dk, dv), stream, check)
+
+
+def gdr_prefill_chunked_cp(q, k, v, a, b, A_log, dt_bias, init_state, out, final_state, T, Hk,
+                           Hv, dk, dv, chunk, nseg, stream=None, check=True):
+    """One sequence cut into at most nseg segments processed side by side on this GPU."""
+    return _call("gdr_prefill_chunked_cp",
+                 (q, k, v, a, b, A_log, dt_bias, init_state, out, final_state),
+                 (T, Hk, Hv, dk, dv, chunk, nseg), stream, check)
 
 
 def gdr_prefill_chunked_f32(q, k, v, a, b, A_log, dt_bias, init_state, out, final_state,

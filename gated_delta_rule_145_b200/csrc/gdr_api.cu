@@ -87,6 +87,31 @@ FwdParams gla(FwdParams p) {
     return p;
 }
 
+// Checks of the segment-map calls: the tensor-core prefill's restrictions (bf16,
+// dk = dv = 128, chunk 32, T >= 1) and the common ones, with no output tensor.
+int check_segment_maps(FwdParams p, const float* phi, const float* nmap) {
+    if (!phi || !nmap) return GDR_ERR_NULL;
+    p.out = const_cast<float*>(nmap);  // stands in for the output in the common checks
+    const int rc = check_common(p, 2);
+    if (rc != GDR_OK) return rc;
+    if (!aligned(phi, 16) || !aligned(nmap, 16)) return GDR_ERR_ALIGN;
+    if (p.chunk != 32 || p.dk != 128 || p.dv != 128 || p.T < 1) return GDR_ERR_UNSUPPORTED;
+    return GDR_OK;
+}
+
+// N (the run from S = 0) into nmap, then Phi (from S = I with v = 0) into phi; no outputs.
+cudaError_t segment_maps(FwdParams p, float* phi, float* nmap, cudaStream_t stream) {
+    p.init_state = nullptr;
+    p.out = nullptr;
+    p.final_state = nmap;
+    cudaError_t e = gdr::launch_prefill_tc(p, stream);
+    if (e != cudaSuccess) return e;
+    p.v_zero = 1;
+    p.init_identity = 1;
+    p.final_state = phi;
+    return gdr::launch_prefill_tc(p, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -116,6 +141,74 @@ int gdr_prefill_chunked_noalloc(const void* q, const void* k, const void* v, con
     void* ws = nullptr;
     if (gdr::noalloc_scratch(&ws) != cudaSuccess) return GDR_ERR_CUDA;
     return to_status(gdr::launch_prefill_tc_ws(p, ws, (cudaStream_t)stream));
+}
+
+int gdr_prefill_segment_maps(const void* q, const void* k, const void* v, const void* a,
+                             const void* b, const float* A_log, const float* dt_bias, float* phi,
+                             float* nmap, const int32_t* cu_seqlens, int B, int T, int Hk, int Hv,
+                             int dk, int dv, int chunk, gdr_stream_t stream) {
+    const FwdParams p = make_params(q, k, v, a, b, A_log, dt_bias, nullptr, nullptr, nullptr,
+                                    cu_seqlens, B, T, Hk, Hv, dk, dv, chunk, InType::BF16);
+    const int rc = check_segment_maps(p, phi, nmap);
+    if (rc != GDR_OK) return rc;
+    return to_status(segment_maps(p, phi, nmap, (cudaStream_t)stream));
+}
+
+int gdr_segment_combine(const float* phi, const float* nmap, const float* init_state,
+                        float* seg_init, float* final_state, int G, int Hv, int dk, int dv,
+                        gdr_stream_t stream) {
+    if (!phi || !nmap) return GDR_ERR_NULL;
+    if (G < 1 || Hv < 1 || (long long)Hv * 4 > 0x7fffffffLL) return GDR_ERR_SHAPE;
+    if (dk != 128 || dv != 128) return GDR_ERR_UNSUPPORTED;
+    if (!aligned(phi, 16) || !aligned(nmap, 16) || !aligned(init_state, 16) ||
+        !aligned(seg_init, 16) || !aligned(final_state, 16))
+        return GDR_ERR_ALIGN;
+    return to_status(gdr::launch_segment_combine(phi, nmap, init_state, seg_init, final_state, G,
+                                                 Hv, dk, (cudaStream_t)stream));
+}
+
+int gdr_prefill_chunked_cp(const void* q, const void* k, const void* v, const void* a,
+                           const void* b, const float* A_log, const float* dt_bias,
+                           const float* init_state, float* out, float* final_state, int T,
+                           int Hk, int Hv, int dk, int dv, int chunk, int nseg,
+                           gdr_stream_t stream) {
+    FwdParams p = make_params(q, k, v, a, b, A_log, dt_bias, init_state, out, final_state,
+                              nullptr, 1, T, Hk, Hv, dk, dv, chunk, InType::BF16);
+    int rc = check_common(p, 2);
+    if (rc != GDR_OK) return rc;
+    if (nseg < 1) return GDR_ERR_SHAPE;
+    if (p.chunk != 32 || p.dk != 128 || p.dv != 128 || p.T < 1) return GDR_ERR_UNSUPPORTED;
+    // chunk-aligned segments of L tokens; G <= nseg of them cover T
+    const long long per = ((long long)T + nseg - 1) / nseg;
+    const int L = (int)((per + 31) / 32 * 32);
+    const int G = (int)(((long long)T + L - 1) / L);
+    const cudaStream_t st = (cudaStream_t)stream;
+    const size_t mat = (size_t)Hv * 128 * 128 * sizeof(float);  // one map per segment
+    const size_t cu_bytes = ((size_t)(G + 1) * sizeof(int32_t) + 255) / 256 * 256;
+    void* ws = nullptr;
+    cudaError_t e = gdr::workspace_alloc(&ws, cu_bytes + 3 * (size_t)G * mat, st);
+    if (e != cudaSuccess) return to_status(e);
+    int32_t* cu = static_cast<int32_t*>(ws);
+    float* phi = reinterpret_cast<float*>(static_cast<char*>(ws) + cu_bytes);
+    float* nmap = reinterpret_cast<float*>(reinterpret_cast<char*>(phi) + (size_t)G * mat);
+    float* seg_init = reinterpret_cast<float*>(reinterpret_cast<char*>(nmap) + (size_t)G * mat);
+    // the segments side by side as the sequences of a packed batch
+    FwdParams sp = p;
+    sp.cu_seqlens = cu;
+    sp.nseq = G;
+    e = gdr::launch_segment_bounds(cu, G, L, T, st);
+    if (e == cudaSuccess) e = segment_maps(sp, phi, nmap, st);
+    if (e == cudaSuccess)
+        e = gdr::launch_segment_combine(phi, nmap, init_state, seg_init, final_state, G, Hv, 128,
+                                        st);
+    if (e == cudaSuccess) {
+        sp.init_state = seg_init;
+        sp.out = out;
+        sp.final_state = nullptr;
+        e = gdr::launch_prefill_tc(sp, st);
+    }
+    const cudaError_t f = cudaFreeAsync(ws, st);
+    return to_status(e != cudaSuccess ? e : f);
 }
 
 int gdr_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,

@@ -21,6 +21,10 @@ struct FwdParams {
     // 1: the gated delta rule; 0: its erase=False special case, gated linear attention
     // (delta = beta v, no k^T S term)
     int erase = 1;
+    // Segment maps (tensor-core prefill only): v_zero runs the rule with v = 0 (v is not
+    // read), init_identity starts every sequence from S = I (dk = dv; init_state is not
+    // read); with out == nullptr no output is written.
+    int v_zero = 0, init_identity = 0;
 };
 
 // Sequential recurrence (decode step and recurrent prefill); recurrent.cu.
@@ -54,6 +58,16 @@ cudaError_t launch_gated_rmsnorm(const float* o, const void* z, bool z_f32, cons
 
 // The fixed scratch area of the no-allocation prefill entry point: its size, and its
 // device address on the current device (looked up once per device); noalloc.cu.
+// Composition of per-segment state maps, and segment boundaries of one sequence cut into
+// G segments of L tokens; segments.cu.
+cudaError_t launch_segment_combine(const float* phi, const float* nmap, const float* init,
+                                   float* seg_init, float* final_state, int G, int Hv, int d,
+                                   cudaStream_t stream);
+cudaError_t launch_segment_bounds(int32_t* cu, int G, int L, int T, cudaStream_t stream);
+
+// The library's stream-ordered workspace pool (prefill_tc.cu).
+cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
+
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** ptr);
 

@@ -2,9 +2,9 @@
 // tensor cores (tcgen05 with accumulators in tensor memory, operands fed by TMA).
 //
 // Sources: Mila "GatedDeltaRule.ixx File Reference", Detailed Description (the step, the
-// gates, the normalisation; prefill runs the chunked UT-transform form with one
-// triangular solve per 32 steps); tessera PR #77 summary, "What landed" (the chunked
-// form's only non-GEMM step is the (I + A)^-1 forward substitution).
+// gates, the normalisation; prefill uses the chunked UT-transform form with one
+// triangular solve per 32 tokens); tessera PR #77 summary, "What landed" (in the
+// chunked form everything but the forward substitution for (I + A)^-1 is a product).
 //
 // Algebra.  Chunk c holds C = 32 tokens; S_c is the state at its start; K_c, Q_c, V_c are
 // the raw bf16 rows; r_k, r_q the inverse row norms (r_q including 1/sqrt(dk)); G the
@@ -543,6 +543,7 @@ struct SpCtx {
 };
 
 // ------------------------------------------------------------------- loads (warp 17)
+template <bool HAS_V>
 __device__ void load_role(SpSmem& sm, const SpCtx& x, int lane, const CUtensorMap* tm_q,
                           const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
     int armed = -2;  // last step whose loads were issued
@@ -554,7 +555,8 @@ __device__ void load_role(SpSmem& sm, const SpCtx& x, int lane, const CUtensorMa
         if (use > 0 && !warp_wait(&sm.abort, &sm.step_empty[r], (uint32_t)(use - 1) & 1u)) break;
         if (lane == 0) {
             const bool next = b + 1 < x.n;
-            const uint32_t bytes = (b >= 0 ? 4u : 2u) * 4096u + (next ? 4096u + 6u * IMG : 0u) +
+            const uint32_t bytes = (b >= 0 ? 4u : 2u) * 4096u +
+                                   (next ? (HAS_V ? 4096u : 0u) + 6u * IMG : 0u) +
                                    (b >= 0 ? 2u * IMG : 0u);
             uint64_t* bar = &sm.step_full[r];
             mbar_arrive_expect_tx(bar, bytes);
@@ -567,7 +569,7 @@ __device__ void load_role(SpSmem& sm, const SpCtx& x, int lane, const CUtensorMa
             }
             SpSmem::Slot& sl = sm.slot[r];
             if (next) {
-                tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, y1, bar);
+                if (HAS_V) tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, y1, bar);
                 const uint8_t* nx = x.record(b + 1);
                 bulk_load(sl.wt[0], nx + rec::OFF_WT, IMG, bar);
                 bulk_load(sl.wt[1], nx + rec::OFF_WT + IMG, IMG, bar);
@@ -597,6 +599,7 @@ __device__ void load_role(SpSmem& sm, const SpCtx& x, int lane, const CUtensorMa
 // covers only its own warp's products; the orderings that cross warps are noted below.
 
 // Delta chain, warp 18.  Step b: acc2 = U_{b+1} + [M_{b+1}; P_b] Delta_b + Wt_{b+1} Y_{b+1}.
+template <bool HAS_V>
 __device__ void chain_role(SpSmem& sm, const SpCtx& x, int lane) {
     const uint32_t id96 = idesc_bf16(64, 2 * NT, 0, 1);
     const uint32_t id48 = idesc_bf16(64, NT, 0, 1);
@@ -618,7 +621,7 @@ __device__ void chain_role(SpSmem& sm, const SpCtx& x, int lane) {
         // acc2[x2] was last read in step b - 2: d_ready phase b - 1, waited in step b - 1
         if (!warp_wait(ab, &sm.step_full[r], (uint32_t)use & 1u)) break;
         tc_fence_after();
-        if (nd) {
+        if (nd && HAS_V) {
             // U: [-Tb_{b+1}; 0] (hi -> columns 0-47, lo -> 48-95) V_{b+1}
             if (leader) {
 #pragma unroll
@@ -639,7 +642,7 @@ __device__ void chain_role(SpSmem& sm, const SpCtx& x, int lane) {
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks)
                     mma_bf16(t2, dadd(d_mp, r * SLOT + ks * 256), dadd(bd, ks * 256), id96,
-                             nd ? 1u : (uint32_t)(ks > 0));
+                             (nd && HAS_V) ? 1u : (uint32_t)(ks > 0));
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks)
                     mma_bf16(t2, dadd(d_mp, r * SLOT + 4096 + ks * 256), dadd(bd, ks * 256), id48, 1);
@@ -654,7 +657,8 @@ __device__ void chain_role(SpSmem& sm, const SpCtx& x, int lane) {
                 const uint64_t by = dadd(d_y, ((b + 1) & 1) * DBUF);
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks)
-                    mma_bf16(t2, dadd(d_wt, r * SLOT + ks * 256), dadd(by, ks * 256), id96, 1);
+                    mma_bf16(t2, dadd(d_wt, r * SLOT + ks * 256), dadd(by, ks * 256), id96,
+                             (HAS_V || b >= 0) ? 1u : (uint32_t)(ks > 0));
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks)
                     mma_bf16(t2, dadd(d_wt, r * SLOT + 4096 + ks * 256), dadd(by, ks * 256), id48, 1);
@@ -745,6 +749,8 @@ drain:
 }
 
 // ------------------------------------------------------------ S group (warps 0-7)
+// INIT_EYE: S_0 = I (else init_state, or zeros without one)
+template <bool INIT_EYE>
 __device__ void s_role(SpSmem& sm, const SpCtx& x, int warp, int lane, const float* init_state,
                        float* final_state) {
     const int q = warp & 3, ch = warp >> 2;
@@ -758,7 +764,13 @@ __device__ void s_role(SpSmem& sm, const SpCtx& x, int warp, int lane, const flo
 #pragma unroll
     for (int j = 0; j < 24; j += 4) {
         float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (init_state && j < nvalid) t = *reinterpret_cast<const float4*>(init_state + srow + j);
+        if (INIT_EYE) {
+            const int c = x.col0 + j0 + j;  // S_0 = I: row k has its 1 in column k
+            t = make_float4(c == k ? 1.f : 0.f, c + 1 == k ? 1.f : 0.f, c + 2 == k ? 1.f : 0.f,
+                            c + 3 == k ? 1.f : 0.f);
+        } else if (init_state && j < nvalid) {
+            t = *reinterpret_cast<const float4*>(init_state + srow + j);
+        }
         Sm[j] = t.x; Sm[j + 1] = t.y; Sm[j + 2] = t.z; Sm[j + 3] = t.w;
     }
     put24(sm.s_op, LO, k, 3 * ch, DK, Sm);
@@ -842,6 +854,8 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
 }
 
 // ---------------------------------------------- output epilogue (warps 10, 11, 14, 15)
+// WRITE_OUT = false: the accumulators are consumed, nothing is stored
+template <bool WRITE_OUT>
 __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __restrict__ out) {
     const int q = warp & 3, ch = (warp - 8) >> 2;
     const int i = 16 * (q - 2) + lane;  // chunk position (valid for lane < 16)
@@ -871,7 +885,7 @@ __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __
         tc_fence_before();
         mbar_arrive(&sm.d_ready);
         const long long c0 = x.t0 + (long long)b * C;
-        if (lane < 16 && c0 + i < x.t1) {
+        if (WRITE_OUT && lane < 16 && c0 + i < x.t1) {
             float* op = out + ((size_t)(c0 + i) * x.Hv + x.h) * DV + x.col0 + j0;
 #pragma unroll
             for (int j = 0; j < 24; j += 4)
@@ -883,6 +897,10 @@ __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __
     }
 }
 
+// Instantiations: <true, true> the prefill; <true, false> a segment's N map (the run from
+// S = 0, no outputs); <false, false> its Phi map (v = 0, so V is neither loaded nor
+// multiplied; S_0 = I; no outputs).
+template <bool HAS_V, bool WRITE_OUT>
 __global__ void __launch_bounds__(SP_THREADS, 1)
 state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const uint8_t* __restrict__ ws,
@@ -907,10 +925,14 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (x.n == 0) {  // empty sequence: the final state is the initial one
         if (final_state && tid < DK) {
             const size_t row = (((size_t)x.s * Hv + x.h) * DK + tid) * DV + x.col0;
-            for (int j = 0; j < x.ncols; j += 4)
+            for (int j = 0; j < x.ncols; j += 4) {
+                const int c = x.col0 + j;
                 *reinterpret_cast<float4*>(final_state + row + j) =
-                    init_state ? *reinterpret_cast<const float4*>(init_state + row + j)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                    !HAS_V ? make_float4(c == tid ? 1.f : 0.f, c + 1 == tid ? 1.f : 0.f,
+                                             c + 2 == tid ? 1.f : 0.f, c + 3 == tid ? 1.f : 0.f)
+                    : init_state ? *reinterpret_cast<const float4*>(init_state + row + j)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
         return;
     }
@@ -958,13 +980,13 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     x.tmem = sm.tmem_base;
 
     if (warp < 8)
-        s_role(sm, x, warp, lane, init_state, final_state);
+        s_role<!HAS_V>(sm, x, warp, lane, init_state, final_state);
     else if (warp < 16)
-        ((warp & 3) < 2) ? d_role(sm, x, warp, lane) : o_role(sm, x, warp, lane, out);
+        ((warp & 3) < 2) ? d_role(sm, x, warp, lane) : o_role<WRITE_OUT>(sm, x, warp, lane, out);
     else if (warp == 17)
-        load_role(sm, x, lane, &tm_q, &tm_k, &tm_v);
+        load_role<HAS_V>(sm, x, lane, &tm_q, &tm_k, &tm_v);
     else if (warp == 18)
-        chain_role(sm, x, lane);
+        chain_role<HAS_V>(sm, x, lane);
     else if (warp == 19)
         state_mma_role(sm, x, lane);
 
@@ -1029,24 +1051,30 @@ cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stre
     const long long tokens = p.cu_seqlens ? (long long)p.T : (long long)p.nseq * p.T;
     if (tokens <= 0 || tokens >= (1LL << 31) - 64) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
+    // with v = 0 the V map is never used; it is built over k (a valid address of the
+    // same row count) only so that every parameter is a well-formed map
     if (!make_bf16_map(&mq, p.q, (uint64_t)p.Hk * DK, tokens) ||
         !make_bf16_map(&mk, p.k, (uint64_t)p.Hk * DK, tokens) ||
-        !make_bf16_map(&mv, p.v, (uint64_t)p.Hv * DV, tokens))
+        !make_bf16_map(&mv, p.v_zero ? p.k : p.v, (uint64_t)(p.v_zero ? p.Hk * DK : p.Hv * DV),
+                       tokens))
         return cudaErrorInvalidValue;
     const long long nrec = rec::max_records(p.cu_seqlens != nullptr, p.nseq, p.T);
     cudaError_t e = cudaFuncSetAttribute(intra_chunk_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(PrepSmem));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(SpSmem));
+    // the Phi pass is v = 0 from S = I without outputs; the N pass has no outputs
+    if (p.v_zero != p.init_identity || (p.v_zero && p.out)) return cudaErrorNotSupported;
+    auto* spk = p.v_zero ? state_pass_kernel<false, false>
+                         : (p.out ? state_pass_kernel<true, true> : state_pass_kernel<true, false>);
+    e = cudaFuncSetAttribute(spk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SpSmem));
     if (e != cudaSuccess) return e;
     intra_chunk_kernel<<<(unsigned)(nrec * p.Hv), PREP_THREADS, sizeof(PrepSmem), stream>>>(
         mq, mk, (const __nv_bfloat16*)p.a, (const __nv_bfloat16*)p.b, p.A_log, p.dt_bias,
         p.cu_seqlens, p.T, p.nseq, p.Hk, p.Hv, p.erase, (uint8_t*)ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    state_pass_kernel<<<(unsigned)(p.nseq * p.Hv * NTILES), SP_THREADS, sizeof(SpSmem), stream>>>(
+    spk<<<(unsigned)(p.nseq * p.Hv * NTILES), SP_THREADS, sizeof(SpSmem), stream>>>(
         mq, mk, mv, (const uint8_t*)ws, p.init_state, p.out, p.final_state, p.cu_seqlens, p.T,
         p.Hk, p.Hv);
     return cudaGetLastError();

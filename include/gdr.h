@@ -12,7 +12,8 @@
  * 1/sqrt(dk), beta_t = sigmoid(b_t) and g_t = -exp(A_log[h]) * softplus(a_t + dt_bias[h]).
  * Value head h reads key/query head h / (Hv / Hk) (consecutive grouping).
  *
- * Two forms of one definition ("TWO FORMS, ONE DEFINITION" on the same page):
+ * Two forms of one definition (same page and section: a sequential form for decode,
+ * a chunked form for prefill):
  *   gdr_prefill_chunked*  -- the chunk-parallel UT-transform form (prefill);
  *   gdr_decode_step*      -- the sequential recurrence on a persistent state (decode);
  *   gdr_prefill_recurrent* -- the sequential recurrence over many tokens in one call.
@@ -72,10 +73,10 @@ typedef void* gdr_stream_t; /* cudaStream_t */
 
 /*
  * Chunked (UT-transform) prefill.  Source: Mila "GatedDeltaRule.ixx File Reference",
- * Detailed Description ("prefill runs the chunked (UT-transform) form ... one
- * triangular solve per 32 steps"); tessera PR #77 summary, "What landed"
- * (gated_delta_rule_chunked: the only non-GEMM step is the (I + A)^-1 forward
- * substitution).
+ * Detailed Description (prefill takes the chunked UT-transform form, with one triangular
+ * solve for every 32 tokens); tessera PR #77 summary, "What landed"
+ * (gated_delta_rule_chunked: apart from the forward substitution for (I + A)^-1,
+ * every step is a matrix product).
  *
  * Dense mode (cu_seqlens == NULL): B sequences of T tokens.
  *   q, k  [B, T, Hk, dk] bf16      v [B, T, Hv, dv] bf16      a, b [B, T, Hv] bf16
@@ -127,6 +128,61 @@ GDR_API int gdr_prefill_chunked_noalloc(const void* q, const void* k, const void
                                         const int32_t* cu_seqlens, int B, int T, int Hk,
                                         int Hv, int dk, int dv, int chunk, gdr_stream_t stream);
 
+/*
+ * Context-parallel prefill: segment maps, their composition, and the one-device form.
+ *
+ * Source: the state update is affine in the state (Mila "GatedDeltaRule.ixx File
+ * Reference", Detailed Description: decay, erase along k, write), so a run of tokens
+ * maps the state at its start to the state at its end as S_end = Phi S_start + N, where
+ * Phi (dk x dk) is the product of the per-token transitions -- the run from S = I with
+ * v = 0 -- and N (dk x dv) is the run from S = 0.  A long sequence cut into segments
+ * (tessera PR #77 summary, on long-context serving) then needs one exchange of the
+ * per-segment (Phi, N): each segment's true start state follows by composing the maps
+ * of the segments before it, and a second pass over each segment from that state gives
+ * its outputs.  These calls take the tensor-core prefill's shapes only: bf16 inputs,
+ * dk = dv = 128, chunk = 32 (anything else returns GDR_ERR_UNSUPPORTED).
+ */
+
+/*
+ * The maps of B segments (dense [B, T] or packed with cu_seqlens, exactly as the
+ * sequences of gdr_prefill_chunked): phi [B, Hv, dk, dk] and nmap [B, Hv, dk, dv], fp32.
+ * No output is written.  Runs the tensor-core prefill twice; T >= 1.
+ */
+GDR_API int gdr_prefill_segment_maps(const void* q, const void* k, const void* v,
+                                     const void* a, const void* b, const float* A_log,
+                                     const float* dt_bias, float* phi, float* nmap,
+                                     const int32_t* cu_seqlens, int B, int T, int Hk, int Hv,
+                                     int dk, int dv, int chunk, gdr_stream_t stream);
+
+/*
+ * Composes the maps of G consecutive segments of one sequence, in order:
+ *   seg_init[0] = init_state (zeros if NULL),
+ *   seg_init[s + 1] = phi[s] seg_init[s] + nmap[s],
+ *   final_state = phi[G - 1] seg_init[G - 1] + nmap[G - 1].
+ * phi, nmap, seg_init [G, Hv, dk, dk]; init_state, final_state [Hv, dk, dv]; fp32.
+ * seg_init and final_state may be NULL (not written).  G >= 1; dk = dv = 128.
+ * seg_init must not alias phi or nmap.
+ */
+GDR_API int gdr_segment_combine(const float* phi, const float* nmap, const float* init_state,
+                                float* seg_init, float* final_state, int G, int Hv, int dk,
+                                int dv, gdr_stream_t stream);
+
+/*
+ * Prefill of ONE sequence of T tokens ([1, T, ...] layouts, init_state and final_state
+ * [1, Hv, dk, dv], nullable as in gdr_prefill_chunked) cut into at most nseg
+ * chunk-aligned segments that run side by side on this device: segment maps, their
+ * composition, then the prefill of every segment from its start state.  Same results as
+ * gdr_prefill_chunked up to rounding; it does about three times the work, in
+ * T / nseg-long chains instead of one T-long chain, which pays when the sequences x
+ * heads of a call leave most of the GPU idle (few heads, long context).  Workspace:
+ * 3 nseg Hv 64 KB from the pool described at the top of this file, plus the prefill's.
+ */
+GDR_API int gdr_prefill_chunked_cp(const void* q, const void* k, const void* v, const void* a,
+                                   const void* b, const float* A_log, const float* dt_bias,
+                                   const float* init_state, float* out, float* final_state,
+                                   int T, int Hk, int Hv, int dk, int dv, int chunk, int nseg,
+                                   gdr_stream_t stream);
+
 /* As gdr_prefill_chunked with fp32 q, k, v, a, b. */
 GDR_API int gdr_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,
                             const float* b, const float* A_log, const float* dt_bias,
@@ -136,8 +192,8 @@ GDR_API int gdr_prefill_chunked_f32(const float* q, const float* k, const float*
 
 /*
  * One decode step on a persistent state, updated in place.  Source: Mila
- * "GatedDeltaRule.ixx File Reference", Detailed Description ("Decode runs the
- * sequential recurrence above").
+ * "GatedDeltaRule.ixx File Reference", Detailed Description (decode uses the
+ * sequential form of the rule).
  *   q, k  [B, Hk, dk] bf16    v [B, Hv, dv] bf16    a, b [B, Hv] bf16
  *   state [B, Hv, dk, dv] fp32, read and overwritten with the new state
  *   out   [B, Hv, dv] fp32
