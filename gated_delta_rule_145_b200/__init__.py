@@ -64,6 +64,7 @@ _SIGS = {
     "gdr_prefill_segment_maps": [_P] * 10 + [_I] * 7 + [_P],
     "gdr_segment_combine": [_P] * 5 + [_I] * 4 + [_P],
     "gdr_prefill_chunked_cp": [_P] * 10 + [_I] * 7 + [_P],
+    "gdr_prefill_chunked_host": [_P] * 10 + [_I] * 8 + [_P],
 }
 
 
@@ -143,6 +144,16 @@ def gdr_prefill_chunked_noalloc(q, k, v, a, b, A_log, dt_bias, init_state, out, 
     return _call("gdr_prefill_chunked_noalloc",
                  (q, k, v, a, b, A_log, dt_bias, init_state, out, final_state, cu_seqlens),
                  (B, T, Hk, Hv, dk, dv, chunk), stream, check)
+
+
+def gdr_prefill_chunked_host(q, k, v, a, b, A_log, dt_bias, init_state, out, final_state, B,
+                             T, Hk, Hv, dk, dv, chunk=32, seg_tokens=0, stream=None,
+                             check=True):
+    """gdr_prefill_chunked from and to HOST buffers (pinned CPU tensors or raw addresses),
+    the copies overlapped with the kernels; complete once `stream` is."""
+    return _call("gdr_prefill_chunked_host",
+                 (q, k, v, a, b, A_log, dt_bias, init_state, out, final_state),
+                 (B, T, Hk, Hv, dk, dv, chunk, seg_tokens), stream, check)
 
 
 def gdr_prefill_segment_maps(q, k, v, a, b, A_log, dt_bias, phi, nmap, cu_seqlens, B, T, Hk,

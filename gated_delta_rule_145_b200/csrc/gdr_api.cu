@@ -211,6 +211,32 @@ int gdr_prefill_chunked_cp(const void* q, const void* k, const void* v, const vo
     return to_status(e != cudaSuccess ? e : f);
 }
 
+int gdr_prefill_chunked_host(const void* q, const void* k, const void* v, const void* a,
+                             const void* b, const float* A_log, const float* dt_bias,
+                             const float* init_state, float* out, float* final_state, int B,
+                             int T, int Hk, int Hv, int dk, int dv, int chunk, int seg_tokens,
+                             gdr_stream_t stream) {
+    if (!A_log || !dt_bias) return GDR_ERR_NULL;
+    if (T > 0 && (!q || !k || !v || !a || !b || !out)) return GDR_ERR_NULL;
+    if (B < 1 || T < 0 || Hk < 1 || Hv < 1 || Hv % Hk != 0 || seg_tokens < 0 ||
+        seg_tokens % 32 != 0 || (long long)B * Hv * 4 > 0x7fffffffLL)
+        return GDR_ERR_SHAPE;
+    if (!head_size_built(dk, dv) || chunk != 32) return GDR_ERR_UNSUPPORTED;
+    // default segment: an eighth of the tokens, at least 256, chunk-aligned
+    int seg = seg_tokens;
+    if (seg == 0) {
+        const long long s8 = ((long long)T + 7) / 8;
+        seg = (int)((s8 < 256 ? 256 : s8) + 31) / 32 * 32;
+    }
+    FwdParams p = make_params(q, k, v, a, b, A_log, dt_bias, init_state, out, final_state,
+                              nullptr, B, T, Hk, Hv, dk, dv, chunk, InType::BF16);
+    int status = GDR_OK;
+    const cudaError_t e = gdr::launch_prefill_host(p, seg, (cudaStream_t)stream,
+                                                   prefill_chunked, &status);
+    if (status != GDR_OK) return status;
+    return to_status(e);
+}
+
 int gdr_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,
                             const float* b, const float* A_log, const float* dt_bias,
                             const float* init_state, float* out, float* final_state,

@@ -65,6 +65,12 @@ cudaError_t launch_segment_combine(const float* phi, const float* nmap, const fl
                                    cudaStream_t stream);
 cudaError_t launch_segment_bounds(int32_t* cu, int G, int L, int T, cudaStream_t stream);
 
+// The chunked prefill from and to host memory in segments of `seg` tokens (a multiple of
+// the chunk), copies overlapped with the kernels; `prefill` runs one device-resident
+// segment and its status lands in *status (0 = OK); host_pipeline.cu.
+cudaError_t launch_prefill_host(const FwdParams& host_params, int seg, cudaStream_t stream,
+                                int (*prefill)(const FwdParams&, cudaStream_t), int* status);
+
 // The library's stream-ordered workspace pool (prefill_tc.cu).
 cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
 

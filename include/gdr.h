@@ -183,6 +183,30 @@ GDR_API int gdr_prefill_chunked_cp(const void* q, const void* k, const void* v, 
                                    int T, int Hk, int Hv, int dk, int dv, int chunk, int nseg,
                                    gdr_stream_t stream);
 
+/*
+ * gdr_prefill_chunked from and to HOST memory (dense layout, bf16 inputs), with the
+ * host-device copies overlapped with the kernels.  q, k, v, a, b, A_log, dt_bias,
+ * init_state (nullable), out and final_state (nullable) are HOST pointers with the
+ * layouts of gdr_prefill_chunked; page-locked (pinned) memory lets the copies run
+ * asynchronously and overlap, pageable memory works but serialises them.
+ *
+ * The tokens are cut into chunk-aligned segments of seg_tokens (0: an eighth of T, at
+ * least 256; otherwise a multiple of 32, else GDR_ERR_SHAPE).  Segment i's inputs are
+ * copied in on a library stream while segment i - 1 computes on `stream` and segment
+ * i - 2's outputs are copied out on another library stream; each sequence's state stays
+ * on the device between segments, so the result is the one-call result up to rounding
+ * (the chunked form restarted at a chunk boundary from the exact fp32 state).  Device
+ * memory: two segments' inputs and outputs plus the states, from the library's pool.
+ * Asynchronous like every call: out and final_state are complete once `stream` is
+ * (the library's streams join it before the call returns).  Calls are serialised per
+ * device while they are enqueued.  dk = dv in {32, 64, 128}; chunk = 32.
+ */
+GDR_API int gdr_prefill_chunked_host(const void* q, const void* k, const void* v,
+                                     const void* a, const void* b, const float* A_log,
+                                     const float* dt_bias, const float* init_state, float* out,
+                                     float* final_state, int B, int T, int Hk, int Hv, int dk,
+                                     int dv, int chunk, int seg_tokens, gdr_stream_t stream);
+
 /* As gdr_prefill_chunked with fp32 q, k, v, a, b. */
 GDR_API int gdr_prefill_chunked_f32(const float* q, const float* k, const float* v, const float* a,
                             const float* b, const float* A_log, const float* dt_bias,
