@@ -129,12 +129,12 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // instructions held by many waiting warps at once congest the shared-memory pipe and slow
 // every other warp's shared-memory, mbarrier and tensor-core traffic.  The polling loop
 // is out of line (one copy serves every call site).
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity);
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity);
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_test(bar, parity)) return true;
     return mbar_wait_slow(bar, parity);
 }
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer();
     for (;;) {
 #pragma unroll 1
