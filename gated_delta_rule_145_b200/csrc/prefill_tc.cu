@@ -480,6 +480,7 @@ struct alignas(1024) SpSmem {
     //   d_ready       Delta_{b+1} written, acc2 of step b read      (chain warp)
     //   dd_ready[x]   D Delta_{b+1} written to dd_op[x]             (state warp)
     uint64_t s_ready, y_ready[2], acc1_free[2], d_ready, dd_ready[2], drain, drain2;
+    uint64_t dd_free[2];  // erase=False form: G3(b) done with dd_op[b % 2] (Delta warps)
     uint32_t tmem_base;
     int abort;
 };
@@ -599,7 +600,7 @@ __device__ void load_role(SpSmem& sm, const SpCtx& x, int lane, const CUtensorMa
 // covers only its own warp's products; the orderings that cross warps are noted below.
 
 // Delta chain, warp 18.  Step b: acc2 = U_{b+1} + [M_{b+1}; P_b] Delta_b + Wt_{b+1} Y_{b+1}.
-template <bool HAS_V>
+template <bool HAS_V, bool ERASE>
 __device__ void chain_role(SpSmem& sm, const SpCtx& x, int lane) {
     const uint32_t id96 = idesc_bf16(64, 2 * NT, 0, 1);
     const uint32_t id48 = idesc_bf16(64, NT, 0, 1);
@@ -649,7 +650,7 @@ __device__ void chain_role(SpSmem& sm, const SpCtx& x, int lane) {
             }
             __syncwarp();
         }
-        if (nd) {
+        if (nd && ERASE) {  // erase=False: Wt = 0, no Y term
             // Y_{b+1}
             if (!warp_wait(ab, &sm.y_ready[(b + 1) & 1], (uint32_t)((b + 1) >> 1) & 1u)) break;
             tc_fence_after();
@@ -683,6 +684,7 @@ __device__ void chain_role(SpSmem& sm, const SpCtx& x, int lane) {
 // acc1 = [K_{b+2}; Q_{b+1}] [S_{b+1} hi | lo].  Y is double-buffered: Y-epi(b) follows
 // this warp's G1a(b), not the chain warp's G1b(b-1), so it writes the other buffer; the
 // buffer it overwrites was read by G1b(b-2), complete before acc2 of step b-2 fired.
+template <bool ERASE>
 __device__ void state_mma_role(SpSmem& sm, const SpCtx& x, int lane) {
     const uint32_t id96 = idesc_bf16(64, 2 * NT, 0, 1);
     const uint32_t id_g3 = idesc_bf16(128, 2 * NT, 1, 1);
@@ -726,6 +728,7 @@ __device__ void state_mma_role(SpSmem& sm, const SpCtx& x, int lane) {
                              dadd(bdd, ks * 256), id_g3, ks > 0);
                 mma_commit(&sm.acc3_full);
                 mma_commit(&sm.step_empty[b % NSTG]);  // pair buffer b - 1 read for the last time
+                if (!ERASE) mma_commit(&sm.dd_free[b & 1]);  // dd_op[b % 2] read
             }
             __syncwarp();
         }
@@ -805,6 +808,9 @@ __device__ void s_role(SpSmem& sm, const SpCtx& x, int warp, int lane, const flo
 }
 
 // -------------------------------------------- Y and Delta epilogues (warps 8, 9, 12, 13)
+// ERASE = false (gated linear attention): no Y, so no Y epilogue; Delta_{b+1} = Tb V does
+// not wait on the state path, and the D Delta buffer is reused only once G3 released it.
+template <bool ERASE>
 __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
     const int q = warp & 3, ch = (warp - 8) >> 2;
     const int r = 16 * q + lane;  // accumulator row (valid for lane < 16)
@@ -820,17 +826,19 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
             gam_next = x.vec(b + 1)[rec::VEC_GAMMA];
             d_next = lane < 16 ? x.vec(b + 2)[rec::VEC_D + r] : 0.f;
         }
-        if (!warp_wait(&sm.abort, &sm.acc1_full[x1], (uint32_t)((b + 1) >> 1) & 1u)) return;
-        tc_fence_after();
         float v[24];
-        ld_sum24(tl + T_ACC1 + 96 * x1 + j0, v);
+        if (ERASE) {
+            if (!warp_wait(&sm.abort, &sm.acc1_full[x1], (uint32_t)((b + 1) >> 1) & 1u)) return;
+            tc_fence_after();
+            ld_sum24(tl + T_ACC1 + 96 * x1 + j0, v);
 #pragma unroll
-        for (int j = 0; j < 24; ++j) v[j] *= gam;
-        if (lane < 16) put24(sm.y_op[(b + 1) & 1], OPB, r, 3 * ch, C, v);
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(&sm.y_ready[(b + 1) & 1]);
-        mbar_arrive(&sm.acc1_free[x1]);
+            for (int j = 0; j < 24; ++j) v[j] *= gam;
+            if (lane < 16) put24(sm.y_op[(b + 1) & 1], OPB, r, 3 * ch, C, v);
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&sm.y_ready[(b + 1) & 1]);
+            mbar_arrive(&sm.acc1_free[x1]);
+        }
         // Delta_{b+1} = -acc2 rows 0-31; D Delta_{b+1}
         if (!warp_wait(&sm.abort, &sm.acc2_full[x1], (uint32_t)((b + 1) >> 1) & 1u)) return;
         tc_fence_after();
@@ -842,10 +850,11 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
             w[j] = d * v[j];
         }
         const int nb = (b + 1) & 1;
-        if (lane < 16) {
-            put24(sm.d_op[nb], OPB, r, 3 * ch, C, v);
-            put24(sm.dd_op[nb], OPB, r, 3 * ch, C, w);
-        }
+        if (lane < 16) put24(sm.d_op[nb], OPB, r, 3 * ch, C, v);
+        // erase=False: dd_op[nb] held D Delta_{b-1}; G3(b-1) releases it (no Y orders it)
+        if (!ERASE && b >= 1 && !warp_wait(&sm.abort, &sm.dd_free[nb], (uint32_t)(((b + 1) >> 1) - 1) & 1u))
+            return;
+        if (lane < 16) put24(sm.dd_op[nb], OPB, r, 3 * ch, C, w);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.d_ready);
@@ -855,7 +864,9 @@ __device__ void d_role(SpSmem& sm, const SpCtx& x, int warp, int lane) {
 
 // ---------------------------------------------- output epilogue (warps 10, 11, 14, 15)
 // WRITE_OUT = false: the accumulators are consumed, nothing is stored
-template <bool WRITE_OUT>
+// ERASE = false: P Delta (acc2) is read before Q S (acc1), so that d_ready, which the Delta
+// chain waits on, does not wait for G1a.
+template <bool WRITE_OUT, bool ERASE>
 __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __restrict__ out) {
     const int q = warp & 3, ch = (warp - 8) >> 2;
     const int i = 16 * (q - 2) + lane;  // chunk position (valid for lane < 16)
@@ -872,18 +883,30 @@ __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __
         const uint32_t ph = (uint32_t)((b + 1) >> 1) & 1u;
         const float e = e_next;
         if (b + 1 < x.n) e_next = lane < 16 ? x.vec(b + 1)[rec::VEC_E + i] : 0.f;
-        if (!warp_wait(&sm.abort, &sm.acc1_full[x1], ph)) return;
-        tc_fence_after();
-        float qs[24];
-        ld_sum24(tl + T_ACC1 + 96 * x1 + j0, qs);
-        tc_fence_before();
-        mbar_arrive(&sm.acc1_free[x1]);
-        if (!warp_wait(&sm.abort, &sm.acc2_full[x1], ph)) return;
-        tc_fence_after();
-        float pd[24];
-        ld_sum24(tl + T_ACC2 + 96 * x1 + j0, pd);
-        tc_fence_before();
-        mbar_arrive(&sm.d_ready);
+        float qs[24], pd[24];
+        if (ERASE) {
+            if (!warp_wait(&sm.abort, &sm.acc1_full[x1], ph)) return;
+            tc_fence_after();
+            ld_sum24(tl + T_ACC1 + 96 * x1 + j0, qs);
+            tc_fence_before();
+            mbar_arrive(&sm.acc1_free[x1]);
+            if (!warp_wait(&sm.abort, &sm.acc2_full[x1], ph)) return;
+            tc_fence_after();
+            ld_sum24(tl + T_ACC2 + 96 * x1 + j0, pd);
+            tc_fence_before();
+            mbar_arrive(&sm.d_ready);
+        } else {
+            if (!warp_wait(&sm.abort, &sm.acc2_full[x1], ph)) return;
+            tc_fence_after();
+            ld_sum24(tl + T_ACC2 + 96 * x1 + j0, pd);
+            tc_fence_before();
+            mbar_arrive(&sm.d_ready);
+            if (!warp_wait(&sm.abort, &sm.acc1_full[x1], ph)) return;
+            tc_fence_after();
+            ld_sum24(tl + T_ACC1 + 96 * x1 + j0, qs);
+            tc_fence_before();
+            mbar_arrive(&sm.acc1_free[x1]);
+        }
         const long long c0 = x.t0 + (long long)b * C;
         if (WRITE_OUT && lane < 16 && c0 + i < x.t1) {
             float* op = out + ((size_t)(c0 + i) * x.Hv + x.h) * DV + x.col0 + j0;
@@ -897,10 +920,11 @@ __device__ void o_role(SpSmem& sm, const SpCtx& x, int warp, int lane, float* __
     }
 }
 
-// Instantiations: <true, true> the prefill; <true, false> a segment's N map (the run from
-// S = 0, no outputs); <false, false> its Phi map (v = 0, so V is neither loaded nor
-// multiplied; S_0 = I; no outputs).
-template <bool HAS_V, bool WRITE_OUT>
+// Instantiations: <true, true, true> the prefill; <true, true, false> the prefill of the
+// erase=False form (gated linear attention); <true, false, true> a segment's N map (the
+// run from S = 0, no outputs); <false, false, true> its Phi map (v = 0, so V is neither
+// loaded nor multiplied; S_0 = I; no outputs).
+template <bool HAS_V, bool WRITE_OUT, bool ERASE>
 __global__ void __launch_bounds__(SP_THREADS, 1)
 state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const uint8_t* __restrict__ ws,
@@ -953,7 +977,8 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(&sm.s_ready, 256);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.y_ready[i], 128);    // Y warps
-            mbar_init(&sm.acc1_free[i], 256);  // Y warps and output warps
+            mbar_init(&sm.acc1_free[i], ERASE ? 256 : 128);  // Y warps (if any) and output warps
+            mbar_init(&sm.dd_free[i], 1);
             mbar_init(&sm.dd_ready[i], 128);   // Delta warps
         }
         mbar_init(&sm.d_ready, 256);           // Delta warps and output warps
@@ -982,13 +1007,14 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp < 8)
         s_role<!HAS_V>(sm, x, warp, lane, init_state, final_state);
     else if (warp < 16)
-        ((warp & 3) < 2) ? d_role(sm, x, warp, lane) : o_role<WRITE_OUT>(sm, x, warp, lane, out);
+        ((warp & 3) < 2) ? d_role<ERASE>(sm, x, warp, lane)
+                         : o_role<WRITE_OUT, ERASE>(sm, x, warp, lane, out);
     else if (warp == 17)
         load_role<HAS_V>(sm, x, lane, &tm_q, &tm_k, &tm_v);
     else if (warp == 18)
-        chain_role<HAS_V>(sm, x, lane);
+        chain_role<HAS_V, ERASE>(sm, x, lane);
     else if (warp == 19)
-        state_mma_role(sm, x, lane);
+        state_mma_role<ERASE>(sm, x, lane);
 
     tc_fence_before();
     __syncthreads();
@@ -1063,10 +1089,14 @@ cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stre
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(PrepSmem));
     if (e != cudaSuccess) return e;
-    // the Phi pass is v = 0 from S = I without outputs; the N pass has no outputs
-    if (p.v_zero != p.init_identity || (p.v_zero && p.out)) return cudaErrorNotSupported;
-    auto* spk = p.v_zero ? state_pass_kernel<false, false>
-                         : (p.out ? state_pass_kernel<true, true> : state_pass_kernel<true, false>);
+    // the Phi pass is v = 0 from S = I without outputs; the N pass has no outputs; both
+    // are of the rule with its erase term
+    if (p.v_zero != p.init_identity || (p.v_zero && p.out) || (!p.erase && !p.out))
+        return cudaErrorNotSupported;
+    auto* spk = p.v_zero ? state_pass_kernel<false, false, true>
+                : !p.out  ? state_pass_kernel<true, false, true>
+                : p.erase ? state_pass_kernel<true, true, true>
+                          : state_pass_kernel<true, true, false>;
     e = cudaFuncSetAttribute(spk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SpSmem));
     if (e != cudaSuccess) return e;
     intra_chunk_kernel<<<(unsigned)(nrec * p.Hv), PREP_THREADS, sizeof(PrepSmem), stream>>>(
