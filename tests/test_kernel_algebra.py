@@ -86,3 +86,27 @@ def test_lookahead_chunk_algebra_matches_the_recurrence(erase, T, C):
                                   inp.init_state[0, h].astype(np.float64), C, erase)
         np.testing.assert_allclose(o, ro[0, :, h], rtol=1e-9, atol=1e-11)
         np.testing.assert_allclose(S, rS[0, h], rtol=1e-9, atol=1e-11)
+
+
+@pytest.mark.parametrize("erase", [True, False])
+def test_decode_step_restatement_matches_the_recurrence(erase):
+    """The decode kernel reads only k^T S and q^T S of the old state: with gamma = e^g,
+    u = k^T S, p = q^T S: delta = beta (v - gamma u) (erase=False: beta v),
+    o = gamma p + (q . k) delta, S' = gamma S + k delta^T (q, k normalised)."""
+    from oracle import oracle
+
+    inp = synth.make_inputs(3, 1, 2, 4, 8, 8, "f32", seed=77, s0_std=0.5)
+    ro, rS = oracle.forward(inp.q, inp.k, inp.v, inp.a, inp.b, inp.A_log, inp.dt_bias,
+                            inp.init_state, erase=erase)
+    qh, kh, g, beta = oracle.prepare(inp.q, inp.k, inp.a, inp.b, inp.A_log, inp.dt_bias)
+    for bq in range(3):
+        for h in range(4):
+            kk, qq = kh[bq, 0, h // 2], qh[bq, 0, h // 2]
+            S = inp.init_state[bq, h].astype(np.float64)
+            gam, bt, v = np.exp(g[bq, 0, h]), beta[bq, 0, h], inp.v[bq, 0, h].astype(np.float64)
+            u, p = kk @ S, qq @ S
+            delta = bt * (v - gam * u) if erase else bt * v
+            o = gam * p + (qq @ kk) * delta
+            S1 = gam * S + np.outer(kk, delta)
+            np.testing.assert_allclose(o, ro[bq, 0, h], rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(S1, rS[bq, h], rtol=1e-10, atol=1e-12)
