@@ -87,9 +87,18 @@ def peaks():
         return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, source="fallback")
 
 
-def kernel_source_hash(name):
-    with open(os.path.join(ROOT, "gated_delta_rule_145_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def kernel_source_hash(name, text=None):
+    """Hash of a kernel source's code: comments and layout removed, so that the recorded
+    traffic stays tied to the code it was measured on, not to its commentary."""
+    if text is None:
+        with open(os.path.join(ROOT, "gated_delta_rule_145_b200", "csrc", name)) as f:
+            text = f.read()
+    import re
+
+    code = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)  # block comments
+    code = re.sub(r"//[^\n]*", " ", code)                 # line comments
+    code = " ".join(code.split())                           # layout
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def recorded_traffic(kernel_file):

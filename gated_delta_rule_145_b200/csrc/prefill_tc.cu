@@ -33,12 +33,17 @@
 //
 // Kernels:
 //   intra_chunk_kernel  one CTA per (chunk, value head), all independent.  Gates, norms,
-//                       the Gram block [K;Q] [K_prev;K]^T on tcgen05, A and P, the forward
-//                       substitution T [diag(w) | diag(beta) | diag(w) K K_prev^T diag(D_prev)]
-//                       = [Wt | Tb | M] with one thread per right-hand-side column, and a
-//                       record of the chunk's operands (chunk_record.h) in the workspace.
+//                       the Gram block [K;Q] [K_prev;K]^T on tcgen05, A and P, T = (I + A)^-1
+//                       by 16 x 16 blocks (the diagonal blocks by forward substitution, one
+//                       column per lane), M = T diag(w) K K_prev^T diag(D_prev), and a record
+//                       of the chunk's operands (chunk_record.h) in the workspace; Wt and Tb
+//                       are column scalings of T applied as the record is written.
 //   state_pass_kernel   one CTA per (sequence, value head, 48-column slice of dv); the
-//                       slice's state stays in registers for the whole sequence.
+//                       slice's state stays in registers for the whole sequence.  A
+//                       template <HAS_V, WRITE_OUT, ERASE>: the prefill, its erase=False
+//                       form (no Y path: Delta = Tb V waits on no state), and the two
+//                       passes that give a segment's state maps (no outputs; v = 0 from
+//                       S = I).
 #include <mutex>
 
 #include "chunk_record.h"
