@@ -139,7 +139,8 @@ int gdr_prefill_chunked_noalloc(const void* q, const void* k, const void* v, con
     if (p.chunk != 32 || p.dk != 128 || p.dv != 128 || p.T < 1) return GDR_ERR_UNSUPPORTED;
     if (gdr::prefill_tc_workspace_bytes(p) > gdr::noalloc_scratch_bytes()) return GDR_ERR_TOO_LARGE;
     void* ws = nullptr;
-    if (gdr::noalloc_scratch(&ws) != cudaSuccess) return GDR_ERR_CUDA;
+    const cudaError_t e = gdr::noalloc_scratch(&ws);
+    if (e != cudaSuccess) return to_status(e);  // the first lookup may fail for lack of memory
     return to_status(gdr::launch_prefill_tc_ws(p, ws, (cudaStream_t)stream));
 }
 

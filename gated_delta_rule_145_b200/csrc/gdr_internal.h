@@ -56,8 +56,6 @@ cudaError_t launch_short_conv_silu(const void* x, const float* w, const float* b
 cudaError_t launch_gated_rmsnorm(const float* o, const void* z, bool z_f32, const float* weight,
                                  float* y, long long rows, int d, float eps, cudaStream_t stream);
 
-// The fixed scratch area of the no-allocation prefill entry point: its size, and its
-// device address on the current device (looked up once per device); noalloc.cu.
 // Composition of per-segment state maps, and segment boundaries of one sequence cut into
 // G segments of L tokens; segments.cu.
 cudaError_t launch_segment_combine(const float* phi, const float* nmap, const float* init,
@@ -74,6 +72,8 @@ cudaError_t launch_prefill_host(const FwdParams& host_params, int seg, cudaStrea
 // The library's stream-ordered workspace pool (prefill_tc.cu).
 cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
 
+// The fixed scratch area of the no-allocation prefill entry point: its size, and its
+// device address on the current device (looked up once per device); noalloc.cu.
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** ptr);
 

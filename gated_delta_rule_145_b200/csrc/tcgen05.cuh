@@ -30,13 +30,7 @@ namespace gdr {
 namespace tc {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-#ifndef GDR_POLL_MODE
-#define GDR_POLL_MODE 0
-#endif
-#ifndef GDR_POLL_SLEEP_NS
-#define GDR_POLL_SLEEP_NS 20
-#endif
-constexpr uint32_t kPollSleepNs = GDR_POLL_SLEEP_NS;
+constexpr uint32_t kPollSleepNs = 20;             // pause between polls of a slow wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -139,14 +133,8 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
     for (;;) {
 #pragma unroll 1
         for (int i = 0; i < 64; ++i) {
-#if GDR_POLL_MODE == 1
-            if (mbar_try_wait(bar, parity)) return true;
-#elif GDR_POLL_MODE == 2
-            if (mbar_test(bar, parity)) return true;
-#else
             __nanosleep(kPollSleepNs);
             if (mbar_test(bar, parity)) return true;
-#endif
         }
         if (globaltimer() - t0 > kWaitLimitNs) return false;
     }

@@ -33,17 +33,21 @@ def head_shard(Hk: int, Hv: int, world: int, rank: int):
 
 def exchange_segment_maps(phi, nmap, group=None):
     """All-gather of every rank's segment map, in rank order: (phi_all, nmap_all) with a
-    leading dimension of world size.  phi and nmap are [1, Hv, dk, dk] tensors on the
-    device of the process group's backend (NCCL: the rank's GPU; gloo: CPU)."""
+    leading dimension of world size, on the device phi and nmap ([1, Hv, dk, dk] and
+    [1, Hv, dk, dv]) live on.  With NCCL the maps travel device to device; a gloo group
+    cannot gather device tensors, so there they are staged through host memory."""
     import torch
     import torch.distributed as dist
 
     world = dist.get_world_size(group)
+    stage = phi.is_cuda and dist.get_backend(group) != "nccl"
     out = []
     for t in (phi, nmap):
-        parts = [torch.empty_like(t) for _ in range(world)]
-        dist.all_gather(parts, t.contiguous(), group=group)
-        out.append(torch.cat(parts, 0))
+        src = t.detach().cpu() if stage else t.contiguous()
+        parts = [torch.empty_like(src) for _ in range(world)]
+        dist.all_gather(parts, src.contiguous(), group=group)
+        res = torch.cat(parts, 0)
+        out.append(res.to(t.device) if stage else res)
     return out[0], out[1]
 
 

@@ -115,7 +115,10 @@ GDR_API int gdr_prefill_chunked(const void* q, const void* k, const void* v, con
  * allocator (no cudaMalloc, cudaMallocAsync or cudaFree).
  *   - The first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any stream
- *     capture on the device.
+ *     capture on the device.  Under lazy module loading (the CUDA default) that lookup
+ *     is also where the library's device code is loaded and the 64 MiB array committed
+ *     on the device, so the first call can fail for lack of device memory
+ *     (GDR_ERR_OOM); later calls allocate nothing.
  *   - Every call on a device shares the same scratch.  The call writes every record it
  *     reads, so nothing needs to start at zero and later calls see no stale state; but
  *     calls that overlap on the GPU (on different streams without ordering between

@@ -66,3 +66,41 @@ def oracle_forward(inp, heads=None, nthreads=None, erase=True):
         S0 = None if S0 is None else S0[:, heads]
     return oracle.forward(q, k, v, a, b, A_log, dt_bias, S0, cu_seqlens=inp.cu_seqlens,
                           nthreads=nthreads, erase=erase)
+
+
+class ParityAccumulator:
+    """max|gpu - oracle| and RMS(oracle) over a whole tensor compared piece by piece (the
+    oracle run on groups of value heads, to bound host memory at the largest sizes); the
+    bar is the same as assert_parity's: max error <= tau * RMS over the whole tensor."""
+
+    def __init__(self, what):
+        self.what, self.err, self.sumsq, self.n = what, 0.0, 0.0, 0
+
+    def add(self, x, ref):
+        x = np.asarray(x, dtype=np.float64)
+        ref = np.asarray(ref, dtype=np.float64)
+        assert np.all(np.isfinite(x)), f"{self.what}: non-finite values"
+        if ref.size:
+            self.err = max(self.err, float(np.max(np.abs(x - ref))))
+            self.sumsq += float(np.sum(ref * ref))
+            self.n += ref.size
+
+    def check(self, tau):
+        rms = (self.sumsq / self.n) ** 0.5 if self.n else 0.0
+        r = self.err / rms if rms > 0 else self.err
+        assert r <= tau, (f"{self.what}: max|err| {self.err:.3e} = {r:.2e} x RMS {rms:.3e} "
+                          f"> {tau:.1e}")
+        return r
+
+
+def check_all_heads(inp, o, S, tau, what, group=12, erase=True):
+    """Every value head of a prefill's outputs o [B,T,Hv,dv] and final states S
+    [Nseq,Hv,dk,dv] (host arrays) against the fp64 oracle, `group` heads per oracle run."""
+    Hv = inp.v.shape[2]
+    acc_o, acc_s = ParityAccumulator(f"{what} o"), ParityAccumulator(f"{what} final state")
+    for h0 in range(0, Hv, group):
+        heads = list(range(h0, min(Hv, h0 + group)))
+        ro, rS = oracle_forward(inp, heads, erase=erase)
+        acc_o.add(o[:, :, heads], ro)
+        acc_s.add(S[:, heads], rS)
+    return acc_o.check(tau), acc_s.check(tau)

@@ -244,3 +244,79 @@ def test_prefill_chunked_cp_matches_oracle(nseg, s0):
     ro, rS = oracle_forward(inp)
     assert_parity(out.cpu().numpy(), ro, TAU["bf16"], f"cp nseg={nseg} o")
     assert_parity(fin.cpu().numpy(), rS, TAU["bf16"], f"cp nseg={nseg} final state")
+
+
+def _cp_rank_worker(rank, world, port, lens, q):
+    """One rank of shard.prefill_context_parallel on GPU 0 under a gloo group: segment
+    `rank` of one sequence in, its outputs and the sequence's final state out (to rank 0)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from gated_delta_rule_145_b200.shard import prefill_context_parallel
+
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        Hk, Hv = 2, 6
+        inp = _one_sequence(sum(lens), Hk, Hv, 128, "bf16", 60, 0.05)
+        d = to_device(inp)
+        t0 = sum(lens[:rank])
+        t1 = t0 + lens[rank]
+        seg = {n: d[n][:, t0:t1].contiguous() for n in ("q", "k", "v", "a", "b")}
+        out = torch.full((1, t1 - t0, Hv, 128), float("nan"), device="cuda")
+        final = prefill_context_parallel(seg["q"], seg["k"], seg["v"], seg["a"], seg["b"],
+                                         d["A_log"], d["dt_bias"], d["init_state"], out, Hk, Hv)
+        torch.cuda.synchronize()
+        status = gdr.gdr_device_status()
+        parts = [None] * world
+        dist.all_gather_object(parts, (out.cpu().numpy(), final.cpu().numpy(), status))
+        if rank == 0:
+            q.put(parts)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_multirank_context_parallel_driver_matches_oracle():
+    """shard.prefill_context_parallel run by two processes on one GPU (gloo exchanges the
+    maps through host memory): the ranks' outputs, concatenated in rank order, and the
+    final state each rank returns equal the oracle's over the whole sequence."""
+    import torch.multiprocessing as mp
+
+    lens = [517, 400]  # ragged segments: 16 chunks + 5 tokens, 12 chunks + 16 tokens
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_rank_worker, args=(r, 2, port, lens, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    import queue
+    import time
+
+    parts, deadline = None, time.time() + 600
+    while parts is None and time.time() < deadline:
+        try:
+            parts = q.get(timeout=5)
+        except queue.Empty:
+            if any(p.exitcode not in (None, 0) for p in procs):
+                break  # a rank failed: stop waiting for the result
+    for p in procs:
+        p.join(timeout=120)
+        if p.is_alive():
+            p.kill()
+        assert p.exitcode == 0
+    assert parts is not None
+    assert all(st == gdr.GDR_OK for _, _, st in parts)
+    from .helpers import oracle_forward
+
+    inp = _one_sequence(sum(lens), 2, 6, 128, "bf16", 60, 0.05)
+    ro, rS = oracle_forward(inp)
+    o = np.concatenate([p[0] for p in parts], axis=1)
+    assert_parity(o, ro, TAU["bf16"], "multi-rank cp o")
+    for r, (_, fin, _) in enumerate(parts):
+        assert_parity(fin, rS, TAU["bf16"], f"multi-rank cp final state (rank {r})")
