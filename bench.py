@@ -283,7 +283,23 @@ def bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth):
     region_ms = _timed(dist, dev, stream, sampler, step, args.steps)
     # two kernels per call: intra-chunk, then state passing
     res = dict(inp=inp, region_ms=region_ms, launches=2 * args.steps,
-               kernel_ms=statistics.mean(s.elapsed_time(e) for s, e in ev))
+               kernel_ms=statistics.mean(s.elapsed_time(e) for s, e in ev),
+               kernel_ms_median=statistics.median(s.elapsed_time(e) for s, e in ev))
+    # the same call timed with the L2 flushed before each call (a 256 MB write between
+    # calls, outside the events): the median per call
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    fl = []
+    for i in range(max(5, min(args.steps, 20))):
+        flush.fill_(i & 255)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        launch(q, k, v, a, b)
+        e1.record(stream)
+        fl.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    res["flushed_median_ms"] = statistics.median(s.elapsed_time(e) for s, e in fl)
+    res["launches"] += 2 * len(fl)
+    del flush
     # the erase=False form (gated linear attention) on the same inputs and kernels
     def gla(_i):
         gdr.gdr_gla_prefill_chunked(q, k, v, a, b, A_log, dt_bias, None, out, fin, None,
@@ -389,6 +405,85 @@ def bench_decode(args, dist, dev, stream, sampler, gdr, synth):
                 kernel_ms=statistics.mean(s.elapsed_time(e) for evs in ev for s, e in evs))
 
 
+def bench_varlen(args, dist, dev, stream, sampler, gdr, synth):
+    """The grouped-key varlen prefill: 8 packed sequences with seeded lengths U[256, 4096],
+    Hk=16 key heads shared by Hv=48 value heads, d=128, chunk 32 (mean per call)."""
+    import torch
+
+    inp = synth.workload(3, seed=1003 + 1000 * dist.rank)
+    d = {n: torch.from_numpy(getattr(inp, n)).to(dev).to(torch.bfloat16)
+         for n in ("q", "k", "v", "a", "b")}
+    A_log = torch.from_numpy(inp.A_log).to(dev)
+    dt_bias = torch.from_numpy(inp.dt_bias).to(dev)
+    cu = torch.from_numpy(inp.cu_seqlens).to(dev)
+    T, nseq = inp.q.shape[1], inp.nseq
+    Hk, Hv = inp.q.shape[2], inp.v.shape[2]
+    out = torch.empty((1, T, Hv, 128), device=dev)
+    fin = torch.empty((nseq, Hv, 128, 128), device=dev)
+    n = max(5, min(args.steps, 20))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+
+    def call(i):
+        ev[i][0].record(stream)
+        gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], A_log, dt_bias, None, out,
+                                fin, cu, nseq, T, Hk, Hv, 128, 128, 32, stream=stream)
+        ev[i][1].record(stream)
+
+    for i in range(3):
+        call(i)
+    ms = _timed(dist, dev, stream, sampler, call, n)
+    kms = statistics.mean(s.elapsed_time(e) for s, e in ev)
+    alg = T * (2 * Hk * 128 * 2 + Hv * 128 * 2 + 2 * Hv * 2 + Hv * 128 * 4) + \
+        nseq * Hv * 128 * 128 * 4
+    lens = np.diff(inp.cu_seqlens).tolist()
+    return dict(workload=f"varlen B={nseq} seqs (lengths {lens}, seeded U[256,4096]) T={T} "
+                         f"Hk={Hk} Hv={Hv} d=128 chunk 32 bf16",
+                tokens=T, ms=ms / n, kernel_ms=kms, alg_bytes=alg, launches=2 * (n + 3))
+
+
+def bench_long(args, dist, dev, stream, sampler, gdr):
+    """Long context: the chunked prefill over B=1, T=65536, Hk=Hv=48, d=128, then 512
+    decode steps from its final state (seeded device-side draws of the same recipe)."""
+    import torch
+
+    g = torch.Generator(device=dev).manual_seed(1004 + 1000 * dist.rank)
+    T, H, nd = 65536, 48, 512
+    r = lambda *shape: torch.randn(shape, device=dev, generator=g).to(torch.bfloat16)
+    x = dict(q=r(1, T + nd, H, 128), k=r(1, T + nd, H, 128), v=r(1, T + nd, H, 128),
+             a=r(1, T + nd, H), b=r(1, T + nd, H))
+    A_log = torch.rand((H,), device=dev, generator=g) * math.log(16.0)
+    dt = torch.exp(torch.rand((H,), device=dev, generator=g) *
+                   (math.log(1e-1) - math.log(1e-3)) + math.log(1e-3))
+    dt_bias = torch.log(torch.expm1(dt))
+    pre = {n: x[n][:, :T] for n in x}
+    dec = {n: x[n][0, T:].contiguous() for n in x}  # [512, ...]: one row per step
+    out = torch.empty((1, T, H, 128), device=dev)
+    S = torch.empty((1, H, 128, 128), device=dev)
+    dout = torch.empty((1, H, 128), device=dev)
+
+    def prefill(_i):
+        gdr.gdr_prefill_chunked(pre["q"], pre["k"], pre["v"], pre["a"], pre["b"], A_log,
+                                dt_bias, None, out, S, None, 1, T, H, H, 128, 128, 32,
+                                stream=stream)
+
+    prefill(0)
+    n = 3
+    pms = _timed(dist, dev, stream, sampler, prefill, n) / n
+
+    def decode(_i):
+        for t in range(nd):
+            gdr.gdr_decode_step(dec["q"][t], dec["k"][t], dec["v"][t], dec["a"][t], dec["b"][t],
+                                A_log, dt_bias, S, dout, 1, H, H, 128, 128, stream=stream)
+
+    dms = _timed(dist, dev, stream, sampler, decode, 1)
+    alg = prefill_alg_bytes(1, T, H, H, 128, 128)
+    return dict(workload=f"long context B=1 T={T} Hk=Hv={H} d=128 chunk 32 bf16, then {nd} "
+                         "decode steps from its final state",
+                prefill_ms=pms, alg_bytes=alg, decode_us_per_step=dms * 1e3 / nd,
+                launches=2 * (n + 1) + nd)
+
+
 def bench_cp(args, dist, dev, stream, sampler, gdr):
     """Context-parallel prefill (segment maps, composition, prefill from each segment's
     start state), two measurements on this GPU:
@@ -480,9 +575,13 @@ def run_ours(args, dist):
         pre = bench_prefill(args, dist, dev, stream, sampler, P, gdr, synth)
     if args.only in (None, "decode"):
         dec = bench_decode(args, dist, dev, stream, sampler, gdr, synth)
-    cpx = None
+    cpx = var = lng = None
     if args.only in (None, "cp"):
         cpx = bench_cp(args, dist, dev, stream, sampler, gdr)
+    if args.only in (None, "varlen"):
+        var = bench_varlen(args, dist, dev, stream, sampler, gdr, synth)
+    if args.only in (None, "long"):
+        lng = bench_long(args, dist, dev, stream, sampler, gdr)
     sampler.stop()
     clocks = sampler.summary()
 
@@ -510,7 +609,9 @@ def run_ours(args, dist):
                     "heads": P["Hv"], "head_dim": P["dk"], "chunk": P["chunk"],
                     "parallelism": f"dp{dist.world} (independent sequences x heads, "
                                    "no collective)",
-                    "l2": "no flush: inputs (302 MB) and outputs (201 MB) exceed the 126 MB L2",
+                    "l2": "value and roofline: no flush between calls (inputs 302 MB and "
+                          "outputs 201 MB exceed the 126 MB L2); flushed_median_ms: 256 MB "
+                          "written before each call",
                 },
                 "roofline": {
                     "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
@@ -518,6 +619,10 @@ def run_ours(args, dist):
                     "traffic": recorded_traffic("prefill_tc.cu"), "peak_source": pk["source"],
                     "alg_bytes_per_launch": alg_b, "alg_flops_per_launch": alg_f,
                     "kernel_ms": round(pre["kernel_ms"], 4),
+                    "kernel_ms_median": round(pre["kernel_ms_median"], 4),
+                    "flushed_median_ms": round(pre["flushed_median_ms"], 4),
+                    "frac_flushed_median": round(alg_b / (pre["flushed_median_ms"] / 1e3) /
+                                                 1e9 / pk["hbm_gbs"], 4),
                     "tensor_frac": round(alg_f / (pre["kernel_ms"] / 1e3) / 1e12 /
                                          pk["bf16_tflops"], 4),
                 },
@@ -554,18 +659,51 @@ def run_ours(args, dist):
             D = DECODE
             dalg = decode_alg_bytes(**D)
             dach = dalg / (dec["kernel_ms"] / 1e3) / 1e9
+            dtraffic = recorded_traffic("recurrent.cu")
+            dcpu = None
+            if dist.world == 1 and not args.no_cpu_baseline and args.only is None:
+                dcpu = decode_cpu_baseline(synth, seconds_hint=args.cpu_seconds / 3)
             result["decode"] = {
                 "workload": DECODE_NAME, "value": round(dec["steps"] / (dec["ms"] / 1e3), 1),
+                "cpu_baseline": dcpu,
                 "unit": "steps/s",
                 "state_gbs": round(decode_state_bytes(**D) * dec["steps"] * dist.world /
                                    (dec["ms"] / 1e3) / 1e9, 1),
                 "ms_per_step": round(dec["ms"] / dec["steps"], 5),
                 "roofline": {"bound": "hbm", "achieved": round(dach, 1), "peak": pk["hbm_gbs"],
                              "unit": "GB/s", "frac": round(dach / pk["hbm_gbs"], 4),
-                             "traffic": recorded_traffic("recurrent.cu"),
+                             "traffic": dtraffic,
                              "alg_bytes_per_launch": dalg,
                              "kernel_ms": round(dec["kernel_ms"], 5)}}
+            if dtraffic:
+                # part of the updated state is still in L2 when the next step reads it:
+                # the DRAM bytes the counters saw per launch, as a fraction of the peak
+                result["decode"]["roofline"]["dram_frac"] = round(
+                    dtraffic / (dec["kernel_ms"] / 1e3) / 1e9 / pk["hbm_gbs"], 4)
             result["gpu_launches"] += dec["steps"]
+        if var is not None:
+            result["gpu_launches"] += var.pop("launches")
+            ach = var["alg_bytes"] / (var["kernel_ms"] / 1e3) / 1e9
+            result["varlen"] = {
+                "workload": var["workload"],
+                "value": round(var["tokens"] * dist.world / (var["ms"] / 1e3), 1),
+                "unit": "tokens/s", "ms_per_step": round(var["ms"], 4),
+                "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4),
+                             "alg_bytes_per_launch": var["alg_bytes"],
+                             "kernel_ms": round(var["kernel_ms"], 4)}}
+        if lng is not None:
+            result["gpu_launches"] += lng.pop("launches")
+            ach = lng["alg_bytes"] / (lng["prefill_ms"] / 1e3) / 1e9
+            result["long"] = {
+                "workload": lng["workload"],
+                "value": round(65536 * dist.world / (lng["prefill_ms"] / 1e3), 1),
+                "unit": "tokens/s", "prefill_ms": round(lng["prefill_ms"], 4),
+                "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4),
+                             "alg_bytes_per_launch": lng["alg_bytes"]},
+                "decode_us_per_step": round(lng["decode_us_per_step"], 2),
+                "decode_note": "B=1: 6.3 MB of state, L2-resident, launch-latency bound"}
         if cpx is not None:
             result["gpu_launches"] += cpx.pop("launches")
             one = cpx["one_gpu"]
@@ -600,6 +738,38 @@ def cpu_baseline_sample(inp, seconds_hint=15.0):
                       f"tokens of the prefill workload, {t:.1f} s wall"}
 
 
+def decode_cpu_baseline(synth, seconds_hint=5.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the decode workload: the first
+    n of its 256 steps for all 64 sequences x 48 heads, on all host cores and on one."""
+    from oracle import oracle
+
+    D = DECODE
+    inp = synth.make_inputs(D["B"], D["steps"], D["Hk"], D["Hv"], D["dk"], D["dv"], "bf16",
+                            seed=1001, s0_std=0.02)
+    cores = oracle.default_threads()
+
+    def run(n, threads):
+        sl = slice(0, n)
+        t0 = time.perf_counter()
+        oracle.forward(inp.q[:, sl], inp.k[:, sl], inp.v[:, sl], inp.a[:, sl], inp.b[:, sl],
+                       inp.A_log, inp.dt_bias, inp.init_state, nthreads=threads)
+        return time.perf_counter() - t0
+
+    res = {}
+    for label, threads in (("all", cores), ("one", 1)):
+        t = run(1, threads)
+        n = int(min(D["steps"], max(1, seconds_hint / max(t, 1e-3))))
+        t = run(n, threads)
+        res[label] = (n / t, n, t)
+    v, n, t = res["all"]
+    v1, n1, t1 = res["one"]
+    return {"value": round(v, 2), "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle, first {n} of 256 decode steps for all 64 x 48 (sequence, "
+                      f"head) states, {t:.1f} s wall",
+            "one_thread": {"value": round(v1, 3), "unit": "steps/s", "cores": 1,
+                           "sample": f"first {n1} steps, {t1:.1f} s wall"}}
+
+
 # ----------------------------------------------------------------- reference arm
 
 
@@ -632,11 +802,15 @@ def run_reference(args, dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same seeded recipe)", "impl": "reference",
-        "config": {"workload": PREFILL_NAME, "global_batch": P["B"], "seq_len": P["T"],
-                   "parallelism": "host threads over heads"},
+        "config": {"workload": PREFILL_NAME if Ts == P["T"] else
+                   PREFILL_NAME + f" (first {Ts} tokens per step)",
+                   "global_batch": P["B"], "seq_len": P["T"], "heads": P["Hv"],
+                   "head_dim": P["dk"], "chunk": P["chunk"],
+                   "parallelism": "host threads over (sequence, head)"},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
                          "kind": "oracle",
-                         "sample": f"fp64 oracle, all 48 heads, first {Ts} tokens per step"},
+                         "sample": f"fp64 oracle, all 48 heads, {Ts} of {P['T']} tokens per "
+                                   "step"},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -650,9 +824,11 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--ref-tokens", type=int, default=128,
-                    help="tokens per reference-arm step (all 48 heads)")
-    ap.add_argument("--only", choices=("prefill", "decode", "cp"), default=None,
+    ap.add_argument("--ref-tokens", type=int, default=PREFILL["T"],
+                    help="tokens per reference-arm step (all 48 heads; default: the whole "
+                         "prefill workload, as our arm)")
+    ap.add_argument("--only", choices=("prefill", "decode", "cp", "varlen", "long"),
+                    default=None,
                     help="time one path only (profiling runs; not the contract line)")
     ap.add_argument("--T", type=int, default=0, help="prefill length override (profiling)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
