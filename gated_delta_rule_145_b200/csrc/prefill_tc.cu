@@ -380,10 +380,11 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     __syncthreads();
     {
-        // Z = A21 T11: thread -> row i, columns 2 cg, 2 cg + 1 (T11 lower triangular)
+        // Z = A21 T11: thread -> row i, columns 2 cg, 2 cg + 1 (unrolled, so that the
+        // shared-memory loads of all 16 terms are in flight together)
         const int i = tid >> 3, j0 = 2 * (tid & 7);
         float z0 = 0.f, z1 = 0.f;
-#pragma unroll 1
+#pragma unroll
         for (int m = 0; m < 16; ++m) {
             const float a_ = sm.f.Am[16 + i][m];
             z0 += a_ * sm.f.u.t.Tm[m][j0];
@@ -394,11 +395,12 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     __syncthreads();
     {
-        // T21 = -T22 Z
+        // T21 = -T22 Z (T22 is stored with its zero upper triangle, so all 16 terms are
+        // summed, unrolled)
         const int i = tid >> 3, j0 = 2 * (tid & 7);
         float t0 = 0.f, t1 = 0.f;
-#pragma unroll 1
-        for (int m = 0; m <= i; ++m) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
             const float t_ = sm.f.u.t.Tm[16 + i][16 + m];
             t0 += t_ * sm.f.u.t.Zm[m][j0];
             t1 += t_ * sm.f.u.t.Zm[m][j0 + 1];
@@ -408,18 +410,24 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     __syncthreads();
     {
-        // M = T R3: thread -> row i, columns 8 cg .. 8 cg + 7 (T lower triangular)
+        // M = T R3: thread -> row i, columns 8 cg .. 8 cg + 7.  T is stored with its zero
+        // upper triangle, so row i sums the terms m < 8 (i / 8 + 1) in unrolled blocks of 8
+        // (the same count for every thread of a warp: a warp holds rows 8 w .. 8 w + 7)
         const int i = tid >> 2, j0 = 8 * (tid & 3);
         float mm[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) mm[q] = 0.f;
 #pragma unroll 1
-        for (int m = 0; m <= i; ++m) {
-            const float t_ = sm.f.u.t.Tm[i][m];
-            const float4 r0 = *reinterpret_cast<const float4*>(&sm.R3[m][j0]);
-            const float4 r1 = *reinterpret_cast<const float4*>(&sm.R3[m][j0 + 4]);
-            mm[0] += t_ * r0.x; mm[1] += t_ * r0.y; mm[2] += t_ * r0.z; mm[3] += t_ * r0.w;
-            mm[4] += t_ * r1.x; mm[5] += t_ * r1.y; mm[6] += t_ * r1.z; mm[7] += t_ * r1.w;
+        for (int m0 = 0; m0 <= i; m0 += 8) {
+#pragma unroll
+            for (int dm = 0; dm < 8; ++dm) {
+                const int m = m0 + dm;
+                const float t_ = sm.f.u.t.Tm[i][m];
+                const float4 r0 = *reinterpret_cast<const float4*>(&sm.R3[m][j0]);
+                const float4 r1 = *reinterpret_cast<const float4*>(&sm.R3[m][j0 + 4]);
+                mm[0] += t_ * r0.x; mm[1] += t_ * r0.y; mm[2] += t_ * r0.z; mm[3] += t_ * r0.w;
+                mm[4] += t_ * r1.x; mm[5] += t_ * r1.y; mm[6] += t_ * r1.z; mm[7] += t_ * r1.w;
+            }
         }
         *reinterpret_cast<float4*>(&sm.f.u.t.Mm[i][j0]) = make_float4(mm[0], mm[1], mm[2], mm[3]);
         *reinterpret_cast<float4*>(&sm.f.u.t.Mm[i][j0 + 4]) = make_float4(mm[4], mm[5], mm[6], mm[7]);
