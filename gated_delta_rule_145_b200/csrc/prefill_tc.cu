@@ -205,6 +205,24 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (tid == 0) atomicExch(&g_tc_status, 2);
         return;
     }
+    // warp 3's global loads for the gates go out first, so that their latency overlaps
+    // the set-up and the tile loads (padding rows: a, b read as 0; their gates are zeroed)
+    __nv_bfloat16 ga{}, gb{}, gpa{}, gpb{};
+    float A_lg = 0.f, dtb = 0.f;
+    if (warp == 3) {
+        A_lg = A_log[h];
+        dtb = dt_bias[h];
+        if (lane < n) {
+            const size_t th = (size_t)(c0 + lane) * Hv + h;
+            ga = a[th];
+            gb = b[th];
+        }
+        if (c > 0) {
+            const size_t th = (size_t)(c0 - C + lane) * Hv + h;
+            gpa = a[th];
+            gpb = b[th];
+        }
+    }
 
     if (tid == 0) {
         mbar_init(&sm.bar_tma, 1);
@@ -234,21 +252,17 @@ intra_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     // ---- gates of this chunk and of the previous one (warp 3); the rest wait for TMA
     if (warp == 3) {
-        const float eA = expf(A_log[h]), dtb = dt_bias[h];
+        const float eA = expf(A_lg);
         float g = 0.f, bt = 0.f;  // padding rows: no decay, no write
-        if (lane < n) {
-            const size_t th = (size_t)(c0 + lane) * Hv + h;
-            gates_fast(__bfloat162float(a[th]), __bfloat162float(b[th]), eA, dtb, g, bt);
-        }
+        if (lane < n) gates_fast(__bfloat162float(ga), __bfloat162float(gb), eA, dtb, g, bt);
         const float Gc = warp_inclusive_scan(g, lane);
         sm.beta[lane] = bt;
         sm.G[lane] = Gc;
         sm.eG[lane] = __expf(Gc);
         float gp = 0.f;
         if (c > 0) {
-            const size_t th = (size_t)(c0 - C + lane) * Hv + h;
             float bp;
-            gates_fast(__bfloat162float(a[th]), __bfloat162float(b[th]), eA, dtb, gp, bp);
+            gates_fast(__bfloat162float(gpa), __bfloat162float(gpb), eA, dtb, gp, bp);
         }
         sm.Gp[lane] = warp_inclusive_scan(gp, lane);
     }
