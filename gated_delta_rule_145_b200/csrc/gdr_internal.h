@@ -40,9 +40,18 @@ cudaError_t launch_chunked_simt(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const FwdParams& p, cudaStream_t stream);
 
 // Bytes of workspace the tensor-core prefill needs for `p`, and the launch on a caller's
-// workspace of at least that size (16-byte aligned); prefill_tc.cu.
+// workspace of at least that size (16-byte aligned); prefill_tc.cu.  It runs the 64-token
+// step kernels of prefill_tc64.cu where they apply (the rule or its erase=False form with
+// outputs), the 32-token step kernels otherwise (the segment-map passes).
 size_t prefill_tc_workspace_bytes(const FwdParams& p);
 cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stream);
+
+// The chunked prefill with the state advanced 64 tokens (two 32-token solve blocks) per
+// serial step: its workspace and launch; prefill_tc64.cu.  cudaErrorNotSupported for the
+// segment-map passes (v = 0, S = I, or no outputs).
+size_t prefill_tc64_workspace_bytes(const FwdParams& p);
+cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t stream);
+int read_and_clear_tc64_status();
 
 // Returns the cached workspace memory of every device to the system; prefill_tc.cu.
 void workspace_release();

@@ -1094,13 +1094,18 @@ void workspace_release() {
         if (ps.made[d]) cudaMemPoolTrimTo(ps.pool[d], 0);
 }
 
+// The 64-token step kernels take the rule and its erase=False form with outputs.
+static bool uses_tc64(const FwdParams& p) { return p.out && !p.v_zero && !p.init_identity; }
+
 size_t prefill_tc_workspace_bytes(const FwdParams& p) {
+    if (uses_tc64(p)) return prefill_tc64_workspace_bytes(p);
     return (size_t)rec::max_records(p.cu_seqlens != nullptr, p.nseq, p.T) * p.Hv * rec::BYTES;
 }
 
 cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stream) {
     if (p.in != InType::BF16 || p.dk != DK || p.dv != DV || p.chunk != C)
         return cudaErrorNotSupported;
+    if (uses_tc64(p)) return launch_prefill_tc64_ws(p, ws, stream);
     const long long tokens = p.cu_seqlens ? (long long)p.T : (long long)p.nseq * p.T;
     if (tokens <= 0 || tokens >= (1LL << 31) - 64) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
@@ -1156,7 +1161,9 @@ int read_and_clear_tc_status() {
         const int zero = 0;
         cudaMemcpyToSymbol(g_tc_status, &zero, sizeof(int));
     }
-    return v;
+    const int v64 = read_and_clear_tc64_status();
+    if (v64 < 0) return -1;
+    return v != 0 ? v : v64;
 }
 
 }  // namespace gdr

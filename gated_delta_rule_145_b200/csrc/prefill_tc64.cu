@@ -1,0 +1,980 @@
+// prefill_tc64.cu -- chunked prefill of the gated delta rule on the sm_100a tensor cores
+// with the state advanced 64 tokens per serial step.
+//
+// Sources: Mila "GatedDeltaRule.ixx File Reference", Detailed Description (the step, the
+// gates, the normalisation; prefill by the chunked UT transform, one triangular solve per
+// 32 tokens); tessera PR #77 summary, "What landed" (apart from the forward substitution
+// for (I + A)^-1 every step of the chunked form is a matrix product).
+//
+// Algebra.  A block of 64 tokens with start state S, raw bf16 rows K, Q, V, inverse row
+// norms r_k, r_q (r_q including 1/sqrt(dk)), cumulative log-decay G over the block
+// (G_i = g_1 + ... + g_i), gamma = e^{G_64}:
+//   A[i,j] = beta_i e^{G_i - G_j} r_k,i r_k,j (K K^T)[i,j]  (j < i)     T = (I + A)^-1
+//   w = beta e^G r_k          B = diag(beta) V - diag(w) K S
+//   Delta = T B               O = diag(E) Q S + P Delta,  E = e^G r_q,
+//   P[i,j] = e^{G_i - G_j} r_q,i r_k,j (Q K^T)[i,j] (j <= i)
+//   S' = gamma S + K^T diag(D) Delta,  D = e^{G_64 - G} r_k.
+// T is built from the two 32-token solves: with T_a, T_b the inverses of the diagonal
+// 32 x 32 blocks (each by 16 x 16 forward substitution and one 16-level coupling),
+// T = [[T_a, 0], [-T_b A_ba T_a, T_b]].  The chunk size of the solve is 32; the state
+// passes over two solve blocks per step.
+//
+// Precision.  As in prefill_tc.cu: products have a raw bf16 operand or split an fp32
+// operand into bf16 hi + lo; derived x derived products take hi*hi + hi*lo + lo*hi.
+//
+// Kernels:
+//   intra64_kernel  one CTA per (64-token block, value head): gates, norms, the Gram
+//                   [K; Q] K^T on tcgen05, A and P, T, and a record holding the operand
+//                   image [-T; P] (128 x 64, hi and lo) and the block's vectors.
+//   state64_kernel  one CTA per (sequence, value head, 48-column slice of dv); per block
+//                   the products G1 = [K; Q] [S hi | lo], Delta = [-T; P] [B hi | lo]
+//                   (rows 0-63: -Delta), G3 = K^T [D Delta hi | lo] and [-T; P] [Delta hi |
+//                   lo] (rows 64-127: P Delta), all M = 128.
+#include "gdr_common.cuh"
+#include "gdr_internal.h"
+#include "tcgen05.cuh"
+#include "tma_map.h"
+
+namespace gdr {
+
+// Set when a bounded wait inside these kernels expired, or shared memory was misaligned
+// (read and cleared by read_and_clear_tc64_status(), reported by gdr_device_status()).
+__device__ int g_tc64_status = 0;
+
+namespace {
+
+using namespace tc;
+
+constexpr int C64 = 64;
+constexpr int DK = 128;
+constexpr int DV = 128;
+
+// ------------------------------------------------------------------ the block record
+// Record (block f, value head h) at ws + (f * Hv + h) * BYTES; blocks are numbered
+// sequence by sequence, each sequence starting a block.
+namespace r64 {
+constexpr uint32_t PART = 16384;            // one 128 x 64 bf16 part of [-T; P]
+constexpr uint32_t OFF_A = 0;               // hi, then lo at + PART
+constexpr uint32_t OFF_VEC = 2 * PART;      // fp32 E[64], D[64], beta[64], w[64], gamma
+constexpr uint32_t VEC_E = 0, VEC_D = 64, VEC_BETA = 128, VEC_W = 192, VEC_GAMMA = 256;
+constexpr uint32_t VEC_BYTES = 1040;        // 257 floats, padded to 16 bytes
+constexpr uint32_t BYTES = 2 * PART + VEC_BYTES;
+
+// Byte offset of row m, K-chunk kc (8 elements) in a K-major no-swizzle image of 8 chunks
+// per row: core matrices of 8 rows x 16 bytes, the 8 chunks of an 8-row group contiguous.
+__host__ __device__ constexpr uint32_t k_off(int m, int kc) {
+    return (uint32_t)((m / 8) * 1024 + kc * 128 + (m % 8) * 16);
+}
+
+__host__ __device__ constexpr long long max_records(bool varlen, int nseq, int T) {
+    return varlen ? ((long long)T + 63LL * nseq) / C64 + 1 : (long long)nseq * ((T + C64 - 1) / C64);
+}
+
+__device__ inline long long block_base(const int32_t* cu, int s, int T) {
+    if (!cu) return (long long)s * ((T + C64 - 1) / C64);
+    long long acc = 0;
+    for (int i = 0; i < s; ++i) acc += (cu[i + 1] - cu[i] + C64 - 1) / C64;
+    return acc;
+}
+
+__device__ inline bool locate(const int32_t* cu, int T, int nseq, long long f, int& s, int& c) {
+    if (!cu) {
+        const long long per = (T + C64 - 1) / C64;
+        if (per == 0 || f >= per * nseq) return false;
+        s = (int)(f / per);
+        c = (int)(f % per);
+        return true;
+    }
+    long long acc = 0;
+    for (int i = 0; i < nseq; ++i) {
+        const long long nb = (cu[i + 1] - cu[i] + C64 - 1) / C64;
+        if (f < acc + nb) {
+            s = i;
+            c = (int)(f - acc);
+            return true;
+        }
+        acc += nb;
+    }
+    return false;
+}
+}  // namespace r64
+
+__device__ __forceinline__ void gates_fast64(float a, float b, float eA, float dt_bias, float& g,
+                                             float& beta) {
+    const float x = a + dt_bias;
+    g = -eA * (fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x))));
+    beta = __frcp_rn(1.f + __expf(-b));
+}
+
+__device__ __forceinline__ float scan32(float x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    return x;
+}
+
+__device__ __forceinline__ uint32_t lane_base64(int warp) { return (uint32_t)((warp & 3) * 32) << 16; }
+__device__ __forceinline__ uint64_t dadd64(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// Sum of squares of the 64 bf16 values in 128 bytes of shared memory.
+__device__ __forceinline__ float sumsq_line(const uint8_t* line) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint4 u = *reinterpret_cast<const uint4*>(line + 16 * j);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            s0 += f.x * f.x;
+            s1 += f.y * f.y;
+        }
+    }
+    return s0 + s1;
+}
+
+// 8 fp32 values (times sc) as one 16-byte chunk of a hi image and of a lo image.
+__device__ __forceinline__ void store_chunk(uint8_t* hi, uint8_t* lo, uint32_t off, const float* x,
+                                            float sc) {
+    uint4 hv, lv;
+    split2(sc * x[0], sc * x[1], hv.x, lv.x);
+    split2(sc * x[2], sc * x[3], hv.y, lv.y);
+    split2(sc * x[4], sc * x[5], hv.z, lv.z);
+    split2(sc * x[6], sc * x[7], hv.w, lv.w);
+    *reinterpret_cast<uint4*>(hi + off) = hv;
+    *reinterpret_cast<uint4*>(lo + off) = lv;
+}
+
+// ================================================================ intra-block kernel
+
+struct alignas(1024) Prep64Smem {
+    union {
+        // per dk half (16 KB): K rows 0-63 | Q rows 64-127, 128-byte rows, 128-byte
+        // swizzle (two TMA boxes of 32 rows each).  Dead once the Gram product and the Q
+        // norms are done; A then takes the space.
+        uint8_t kq[2][16384];
+        float Am[C64][68];
+    };
+    float Tm[C64][68];  // T = (I + A)^-1, stored with its zero upper triangle
+    float Zm[32][36];   // coupling products
+    alignas(16) float beta[C64];
+    alignas(16) float G[C64];   // G of tokens 32-63 still lacks the first half's total
+    alignas(16) float rk[C64];
+    alignas(16) float rq[C64];
+    uint64_t bar_tma, bar_mma;
+    uint32_t tmem;
+};
+static_assert(sizeof(Prep64Smem) <= 57 * 1024, "four intra-block CTAs per SM");
+
+constexpr int PREP64_THREADS = 128;
+
+__global__ void __launch_bounds__(PREP64_THREADS, 4)
+intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+               const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+               const int32_t* __restrict__ cu_seqlens, int T, int nseq, int Hk, int Hv, int erase,
+               uint8_t* __restrict__ ws) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    Prep64Smem& sm = *reinterpret_cast<Prep64Smem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int h = blockIdx.x % Hv;
+    const long long f = blockIdx.x / Hv;
+    int s, c;
+    if (!r64::locate(cu_seqlens, T, nseq, f, s, c)) return;  // past the last block
+    long long t0, t1;
+    seq_range(cu_seqlens, s, T, t0, t1);
+    const long long c0 = t0 + (long long)c * C64;
+    const int n = (int)min((long long)C64, t1 - c0);
+    const int kh = h / (Hv / Hk);
+    uint8_t* rc = ws + ((size_t)f * Hv + h) * r64::BYTES;
+    if ((smem_u32(smem_raw) & 1023u) != 0) {  // swizzled tiles need 1 KB alignment
+        if (tid == 0) atomicExch(&g_tc64_status, 2);
+        return;
+    }
+    // gate inputs: warp 2 tokens 0-31, warp 3 tokens 32-63 (padding rows read nothing)
+    __nv_bfloat16 ga{}, gb{};
+    float A_lg = 0.f, dtb = 0.f;
+    if (warp >= 2) {
+        A_lg = A_log[h];
+        dtb = dt_bias[h];
+        const int i = 32 * (warp - 2) + lane;
+        if (i < n) {
+            const size_t th = (size_t)(c0 + i) * Hv + h;
+            ga = a[th];
+            gb = b[th];
+        }
+    }
+    if (tid == 0) {
+        mbar_init(&sm.bar_tma, 1);
+        mbar_init(&sm.bar_mma, 1);
+        mbar_init_fence();
+        mbar_arrive_expect_tx(&sm.bar_tma, 8u * 4096u);
+        for (int hf = 0; hf < 2; ++hf) {
+            const int x = kh * DK + 64 * hf;
+            tma_load_2d(sm.kq[hf], &tm_k, x, (int)c0, &sm.bar_tma);
+            tma_load_2d(sm.kq[hf] + 4096, &tm_k, x, (int)c0 + 32, &sm.bar_tma);
+            tma_load_2d(sm.kq[hf] + 8192, &tm_q, x, (int)c0, &sm.bar_tma);
+            tma_load_2d(sm.kq[hf] + 12288, &tm_q, x, (int)c0 + 32, &sm.bar_tma);
+        }
+    }
+    if (warp == 0) tmem_alloc(&sm.tmem, 64);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+    if (warp >= 2) {
+        const int i = 32 * (warp - 2) + lane;
+        float g = 0.f, bt = 0.f;  // padding rows: no decay, no write
+        if (i < n) gates_fast64(__bfloat162float(ga), __bfloat162float(gb), expf(A_lg), dtb, g, bt);
+        sm.beta[i] = bt;
+        sm.G[i] = scan32(g, lane);
+    }
+    bool ok = __syncthreads_and(mbar_wait(&sm.bar_tma, 0)) != 0;
+    // ---- Gram [K; Q] K^T  (M = 128, N = 64, K = 128): rows 0-63 K K^T, 64-127 Q K^T
+    if (warp == 0) {
+        if (ok && elect_one()) {
+            const uint32_t base = smem_u32(sm.kq[0]);
+            const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                mma_bf16(tmem, sdesc(base + off, 16, 1024, kSw128),
+                         sdesc(base + off, 16, 1024, kSw128), id, ks > 0);
+            }
+            mma_commit(&sm.bar_mma);
+        }
+        __syncwarp();
+    }
+    // ---- inverse norms of the Q rows (thread pair per row; the swizzle only permutes
+    //      16-byte pieces inside a row, which a sum ignores)
+    if (ok) {
+        const int row = tid >> 1, hf = tid & 1;
+        float ss = sumsq_line(sm.kq[hf] + 8192 + row * 128);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if (hf == 0) sm.rq[row] = rsqrtf(ss + kNormEps) * rsqrtf((float)DK);
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&sm.bar_mma, 0)) != 0;
+    tc_fence_after();
+    // accumulator row 32 w + lane: warps 0, 1 rows of K K^T, warps 2, 3 rows of Q K^T
+    float v[C64];
+    if (ok) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+            tmem_ld16(tmem + lane_base64(warp) + 16 * q4, *reinterpret_cast<float(*)[16]>(&v[16 * q4]));
+        tmem_ld_wait();
+    }
+    if (warp < 2) {  // r_k from the diagonal of K K^T
+        const int i = 32 * warp + lane;
+        float dd = 0.f;
+#pragma unroll
+        for (int j = 0; j < C64; ++j) dd = j == i ? v[j] : dd;
+        sm.rk[i] = rsqrtf(dd + kNormEps);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (!ok) {
+        if (tid == 0) atomicExch(&g_tc64_status, 1);
+        return;
+    }
+    const float G31 = sm.G[31];
+    auto Gf = [&](int j) { return sm.G[j] + (j >= 32 ? G31 : 0.f); };
+
+    // ---- A rows into shared memory (warps 0, 1); P rows straight into the record's
+    //      image rows 64-127 (warps 2, 3)
+    if (warp < 2) {
+        const int i = 32 * warp + lane;
+        const float Gi = Gf(i), fa = erase ? sm.beta[i] * sm.rk[i] : 0.f;
+#pragma unroll
+        for (int j = 0; j < C64; j += 4) {
+            float4 o;
+            float* op = &o.x;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int jj = j + e;
+                const float av = fa * __expf(Gi - Gf(jj)) * sm.rk[jj] * v[jj];
+                op[e] = jj < i ? av : 0.f;
+            }
+            *reinterpret_cast<float4*>(&sm.Am[i][j]) = o;
+        }
+    } else {
+        const int i = 32 * (warp - 2) + lane;
+        const float Gi = Gf(i), fp = sm.rq[i];
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int jj = 8 * kc + e;
+                const float pv = fp * __expf(Gi - Gf(jj)) * sm.rk[jj] * v[jj];
+                p[e] = jj <= i ? pv : 0.f;
+            }
+            store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(C64 + i, kc), p, 1.f);
+        }
+    }
+    __syncthreads();
+
+    // ---- T = (I + A)^-1.  The four diagonal 16 x 16 blocks by forward substitution, one
+    //      column per lane (warps 0 and 1: lanes 0-15 and 16-31 take one block each);
+    //      warps 2 and 3 zero the blocks above the diagonal.
+    if (warp < 2) {
+        const int o = 32 * warp + (lane & 16), j = lane & 15;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float s0 = i == j ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < (i & ~1); m += 2) {
+                const float2 av = *reinterpret_cast<const float2*>(&sm.Am[o + i][o + m]);
+                s0 -= av.x * x[m];
+                s1 -= av.y * x[m + 1];
+            }
+            if (i & 1) s0 -= sm.Am[o + i][o + i - 1] * x[i - 1];
+            x[i] = s0 + s1;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sm.Tm[o + i][o + j] = x[i];
+    } else {
+        // rows 16 bi .. 16 bi + 15, columns right of the diagonal block: 6 blocks
+        for (int e = tid - 64; e < 6 * 256; e += 64) {
+            const int blk = e >> 8, w = e & 255, r = w >> 4, cc = w & 15;
+            // blocks (row band, column band): (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+            const int rb = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int cb = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            sm.Tm[16 * rb + r][16 * cb + cc] = 0.f;
+        }
+    }
+    __syncthreads();
+    {
+        // 16-level coupling inside each 32-token block (its triangular solve):
+        // Z = A[b+16.., b..] T[b.., b..], thread -> (block bi, row i, 4 columns)
+        const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const float a_ = sm.Am[o + 16 + i][o + m];
+            const float4 t4 = *reinterpret_cast<const float4*>(&sm.Tm[o + m][o + jc]);
+            z[0] += a_ * t4.x; z[1] += a_ * t4.y; z[2] += a_ * t4.z; z[3] += a_ * t4.w;
+        }
+        *reinterpret_cast<float4*>(&sm.Zm[16 * bi + i][jc]) = make_float4(z[0], z[1], z[2], z[3]);
+    }
+    __syncthreads();
+    {
+        // T[b+16.., b..] = -T[b+16.., b+16..] Z (the lower diagonal block has its zero
+        // upper triangle stored, so all 16 terms are summed)
+        const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
+        float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const float tv = sm.Tm[o + 16 + i][o + 16 + m];
+            const float4 z4 = *reinterpret_cast<const float4*>(&sm.Zm[16 * bi + m][jc]);
+            t[0] += tv * z4.x; t[1] += tv * z4.y; t[2] += tv * z4.z; t[3] += tv * z4.w;
+        }
+        *reinterpret_cast<float4*>(&sm.Tm[o + 16 + i][o + jc]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+    }
+    __syncthreads();
+    {
+        // 32-level coupling: Z = A_ba T_a (rows 32-63, columns 0-31), thread -> row i,
+        // columns 8 cg .. 8 cg + 7
+        const int i = tid >> 2, j0 = 8 * (tid & 3);
+        float z[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) z[q] = 0.f;
+#pragma unroll 4
+        for (int m = 0; m < 32; ++m) {
+            const float a_ = sm.Am[32 + i][m];
+            const float4 t0v = *reinterpret_cast<const float4*>(&sm.Tm[m][j0]);
+            const float4 t1v = *reinterpret_cast<const float4*>(&sm.Tm[m][j0 + 4]);
+            z[0] += a_ * t0v.x; z[1] += a_ * t0v.y; z[2] += a_ * t0v.z; z[3] += a_ * t0v.w;
+            z[4] += a_ * t1v.x; z[5] += a_ * t1v.y; z[6] += a_ * t1v.z; z[7] += a_ * t1v.w;
+        }
+        *reinterpret_cast<float4*>(&sm.Zm[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
+        *reinterpret_cast<float4*>(&sm.Zm[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
+    }
+    __syncthreads();
+    {
+        // T_ba = -T_b Z
+        const int i = tid >> 2, j0 = 8 * (tid & 3);
+        float t[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) t[q] = 0.f;
+#pragma unroll 4
+        for (int m = 0; m < 32; ++m) {
+            const float tv = sm.Tm[32 + i][32 + m];
+            const float4 z0 = *reinterpret_cast<const float4*>(&sm.Zm[m][j0]);
+            const float4 z1 = *reinterpret_cast<const float4*>(&sm.Zm[m][j0 + 4]);
+            t[0] += tv * z0.x; t[1] += tv * z0.y; t[2] += tv * z0.z; t[3] += tv * z0.w;
+            t[4] += tv * z1.x; t[5] += tv * z1.y; t[6] += tv * z1.z; t[7] += tv * z1.w;
+        }
+        *reinterpret_cast<float4*>(&sm.Tm[32 + i][j0]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+        *reinterpret_cast<float4*>(&sm.Tm[32 + i][j0 + 4]) = make_float4(-t[4], -t[5], -t[6], -t[7]);
+    }
+    __syncthreads();
+    // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int task = tid + PREP64_THREADS * e, row = task >> 3, kc = task & 7;
+        store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(row, kc),
+                    &sm.Tm[row][8 * kc], -1.f);
+    }
+    // ---- vectors
+    if (tid < C64) {
+        const int i = tid;
+        float* vec = reinterpret_cast<float*>(rc + r64::OFF_VEC);
+        const float Gi = Gf(i), GC = Gf(C64 - 1), eG = __expf(Gi);
+        vec[r64::VEC_E + i] = eG * sm.rq[i];
+        vec[r64::VEC_D + i] = __expf(GC - Gi) * sm.rk[i];
+        vec[r64::VEC_BETA + i] = sm.beta[i];
+        vec[r64::VEC_W + i] = erase ? sm.beta[i] * eG * sm.rk[i] : 0.f;
+        if (i == 0) vec[r64::VEC_GAMMA] = __expf(GC);
+    }
+}
+
+// ================================================================= state-passing kernel
+
+constexpr int NT = 48;                      // dv columns per CTA
+constexpr int NTILES = (DV + NT - 1) / NT;  // 3 (the last a third empty)
+constexpr int SP_THREADS = 640;             // 20 warps
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t T_ACC1 = 0;    // 2 x 96, M = 128: rows 0-63 K S, 64-127 Q S ([hi | lo])
+constexpr uint32_t T_ACC2 = 192;  // 96: rows 0-63 -Delta
+constexpr uint32_t T_ACC3 = 288;  // 96: K^T D Delta (state update)
+constexpr uint32_t T_ACC4 = 384;  // 96: rows 64-127 P Delta
+constexpr uint32_t OPB = NT * C64 * 2;  // one K = 64 x N = 48 bf16 operand part (6144 B)
+constexpr int O_PITCH = 52;             // floats: 208 B rows, 16-byte aligned
+
+// Warp roles
+//   0-7            S group: the state slice in registers (row 32 (w % 4) + lane, 24 columns
+//                  per warp half); S <- gamma S + K^T D Delta and the state's hi/lo operand
+//   8, 9, 12, 13   BD group (accumulator rows 0-63): B = diag(beta) V - diag(w) K S and
+//                  Delta, D Delta
+//   10, 11, 14, 15 output group (accumulator rows 64-127): O = E Q S + P Delta, staged in
+//                  shared memory and written by one bulk copy per row segment (per-lane
+//                  stores to rows 24 KB apart would hold up the memory pipe that the
+//                  operand stores of the chain use)
+//   16             loads: TMA tiles [K; Q] and V, the record image [-T; P] and its
+//                  vectors, two-deep ring
+// The S and BD groups read nothing from global memory inside the loop: a named barrier
+// orders memory like membar.cta and so waits for a warp's global loads still in flight.
+//   18             issues Delta, K^T D Delta and P Delta (meets the BD group on BAR_BD);
+//                  P Delta(s) only after G1(s+1) was issued, so that the tensor pipe runs
+//                  the chain's product first
+//   19             issues [K; Q] [S hi | lo] (meets the S group on BAR_S)
+//   17             no role
+struct alignas(1024) Sp64Smem {
+    uint8_t kq[2][32768];   // block s: per dk half (16 KB) K rows 0-63 | Q rows 64-127
+    uint8_t rec[2][32768];  // block s: [-T; P] hi (16 KB), lo (16 KB)
+    uint8_t vt[2][8192];    // block s: V columns col0 .. col0 + 63, 64 rows (128-byte swizzle)
+    float vec[2][260];      // block s: the record's E, D, beta, w, gamma
+    // thread-written MN-major no-swizzle B operands, hi part then lo part along N
+    uint8_t s_op[2 * NT * DK * 2];  // S: K = 128
+    uint8_t b_op[2 * OPB];          // B: K = 64
+    uint8_t d_op[2 * OPB];          // Delta
+    uint8_t dd_op[2 * OPB];         // diag(D) Delta
+    float o_st[C64][O_PITCH];       // output rows of block s (pitch: conflict-free v4 stores)
+    uint64_t full[2], empty[2];
+    uint64_t acc1_full[2], acc1_free[2], acc2_full, g1_issued;
+    uint64_t acc3_full, acc3_free, acc4_full, acc4_free, drain_s, drain_d;
+    uint32_t tmem_base;
+    int abort;
+};
+
+static_assert(sizeof(Sp64Smem) <= 227 * 1024, "one state CTA per SM");
+
+__device__ __forceinline__ bool w64(int* abort, uint64_t* bar, uint32_t parity) {
+    if (mbar_test(bar, parity)) return true;
+    if (*(volatile int*)abort) return false;
+    if (mbar_wait_slow(bar, parity)) return true;
+    atomicExch(abort, 1);
+    return false;
+}
+
+// Named barriers: the S group with the G1 issuing warp; the BD group with the Delta issuing
+// warp.  Every warp of a pair runs every barrier of it, also once the kernel is aborting
+// (its waits then return at once), so a timed-out wait cannot strand a barrier.
+constexpr uint32_t BAR_S = 1, BAR_BD = 2;
+constexpr uint32_t BAR_S_THREADS = 9 * 32, BAR_BD_THREADS = 5 * 32;
+
+__device__ __forceinline__ void gbar(uint32_t id, uint32_t nthreads) {
+    __syncwarp();
+    named_bar(id, nthreads);
+}
+
+__device__ __forceinline__ void warp_arrive64(uint64_t* bar, int lane) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+}
+
+__device__ __forceinline__ uint32_t mn_off64(int k, int g, int krows) {
+    return (uint32_t)(g * (krows / 8) * 128 + k * 16);
+}
+
+// 24 fp32 values (times sc) of K-row k (column groups g0 .. g0 + 2) as the hi and lo parts
+// of an MN-major operand whose lo part starts lo_off bytes after the hi part.
+__device__ __forceinline__ void put24s(uint8_t* op, uint32_t lo_off, int k, int g0, int krows,
+                                       const float (&v)[24], float sc) {
+#pragma unroll
+    for (int g = 0; g < 3; ++g) {
+        uint4 hv, lv;
+        split2(sc * v[8 * g + 0], sc * v[8 * g + 1], hv.x, lv.x);
+        split2(sc * v[8 * g + 2], sc * v[8 * g + 3], hv.y, lv.y);
+        split2(sc * v[8 * g + 4], sc * v[8 * g + 5], hv.z, lv.z);
+        split2(sc * v[8 * g + 6], sc * v[8 * g + 7], hv.w, lv.w);
+        const uint32_t o = mn_off64(k, g0 + g, krows);
+        *reinterpret_cast<uint4*>(op + o) = hv;
+        *reinterpret_cast<uint4*>(op + lo_off + o) = lv;
+    }
+}
+
+// v = sc * v + (hi + lo halves of a [hi | lo] accumulator), 24 columns from taddr.
+__device__ __forceinline__ void ld_acc24s(uint32_t taddr, float sc, float (&v)[24]) {
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        float t[24];
+        tmem_ld16(taddr + NT * part, *reinterpret_cast<float(*)[16]>(&t[0]));
+        tmem_ld8(taddr + NT * part + 16, &t[16]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 24; ++i) v[i] = (part == 0 ? sc * v[i] : v[i]) + t[i];
+    }
+}
+
+struct Sp64Ctx {
+    int s, h, kh, Hv, col0, n;
+    long long t0, t1, rbase;
+    const uint8_t* ws;
+    uint32_t tmem;
+    __device__ const float* vec(int blk) const {
+        return reinterpret_cast<const float*>(ws + ((size_t)(rbase + blk) * Hv + h) * r64::BYTES +
+                                              r64::OFF_VEC);
+    }
+    __device__ const uint8_t* record(int blk) const {
+        return ws + ((size_t)(rbase + blk) * Hv + h) * r64::BYTES;
+    }
+};
+
+// ------------------------------------------------------------------- loads (warp 16)
+__device__ void load64_role(Sp64Smem& sm, const Sp64Ctx& x, int lane, const CUtensorMap* tm_q,
+                            const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
+    int armed = -1;
+    for (int s = 0; s < x.n; ++s) {
+        const int r = s & 1, use = s >> 1;
+        if (use > 0 && !w64(&sm.abort, &sm.empty[r], (uint32_t)(use - 1) & 1u)) break;
+        if (lane == 0) {
+            uint64_t* bar = &sm.full[r];
+            mbar_arrive_expect_tx(bar, 10u * 4096u + 2u * r64::PART + r64::VEC_BYTES);
+            const int y = (int)(x.t0 + (long long)s * C64);
+            for (int hf = 0; hf < 2; ++hf) {
+                const int xx = x.kh * DK + 64 * hf;
+                uint8_t* base = sm.kq[r] + 16384 * hf;
+                tma_load_2d(base, tm_k, xx, y, bar);
+                tma_load_2d(base + 4096, tm_k, xx, y + 32, bar);
+                tma_load_2d(base + 8192, tm_q, xx, y, bar);
+                tma_load_2d(base + 12288, tm_q, xx, y + 32, bar);
+            }
+            tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, y, bar);
+            tma_load_2d(sm.vt[r] + 4096, tm_v, x.h * DV + x.col0, y + 32, bar);
+            const uint8_t* rc = x.record(s);
+            bulk_load(sm.rec[r], rc + r64::OFF_A, r64::PART, bar);
+            bulk_load(sm.rec[r] + r64::PART, rc + r64::OFF_A + r64::PART, r64::PART, bar);
+            bulk_load(sm.vec[r], rc + r64::OFF_VEC, r64::VEC_BYTES, bar);
+        }
+        __syncwarp();
+        armed = s;
+    }
+    // every copy this warp started has landed before the CTA may exit
+    for (int s = max(0, armed - 1); s <= armed; ++s) mbar_wait(&sm.full[s & 1], (uint32_t)(s >> 1) & 1u);
+    __syncwarp();
+}
+
+// ---------------------------------------------------------- issuing warps (18, 19)
+// Warp 19: G1(s) = [K_s; Q_s] [S_s hi | lo] into acc1[s & 1].
+__device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
+    const uint32_t id96 = idesc_bf16(128, 2 * NT, 0, 1);
+    const uint64_t d_kq = sdesc(smem_u32(sm.kq[0]), 16, 1024, kSw128);  // [K;Q] K-major
+    const uint64_t d_s = sdesc(smem_u32(sm.s_op), 128, 2048, kSwNone);
+    const bool leader = lane == 0;
+    int* ab = &sm.abort;
+    bool live = true;
+    for (int s = 0; s < x.n; ++s) {
+        const int r = s & 1, x1 = s & 1;
+        gbar(BAR_S, BAR_S_THREADS);  // S_s written
+        if (leader && live) {
+            live = w64(ab, &sm.full[r], (uint32_t)(s >> 1) & 1u) &&        // tiles of s
+                   (s < 2 || w64(ab, &sm.acc1_free[x1], (uint32_t)((s >> 1) - 1) & 1u));
+            if (live) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16(x.tmem + T_ACC1 + 96 * x1,
+                             dadd64(d_kq, r * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32),
+                             dadd64(d_s, ks * 256), id96, ks > 0);
+                mma_commit(&sm.acc1_full[x1]);
+                mma_commit(&sm.empty[r]);
+                if (s >= 1) mbar_arrive(&sm.g1_issued);
+            }
+        }
+        __syncwarp();
+    }
+    if (leader) {
+        mma_commit(&sm.drain_s);
+        mbar_wait(&sm.drain_s, 0);
+    }
+    __syncwarp();
+}
+
+// Warp 18: Delta(s) = [-T; P] [B hi | lo] into acc2; G3(s) = K_s^T [D Delta hi | lo] into
+// acc3; [-T; P] [Delta hi | lo] into acc4.
+__device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
+    const uint32_t id96 = idesc_bf16(128, 2 * NT, 0, 1);
+    const uint32_t id48 = idesc_bf16(128, NT, 0, 1);
+    const uint32_t id_g3 = idesc_bf16(128, 2 * NT, 1, 1);
+    const uint64_t d_rec = sdesc(smem_u32(sm.rec[0]), 128, 1024, kSwNone);   // [-T; P] K-major
+    const uint64_t d_kt = sdesc(smem_u32(sm.kq[0]), 16384, 1024, kSw128);    // K^T MN-major
+    const uint64_t d_b = sdesc(smem_u32(sm.b_op), 128, 1024, kSwNone);
+    const uint64_t d_d = sdesc(smem_u32(sm.d_op), 128, 1024, kSwNone);
+    const uint64_t d_dd = sdesc(smem_u32(sm.dd_op), 128, 1024, kSwNone);
+    const bool leader = lane == 0;
+    int* ab = &sm.abort;
+    // [-T; P] (hi, lo) times an [X hi | X lo] operand: hi x [hi | lo] (N = 96) + lo x hi
+    auto tp_product = [&](int r, uint32_t dcol, uint64_t dx) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(x.tmem + dcol, dadd64(d_rec, r * 32768 + ks * 256), dadd64(dx, ks * 256), id96,
+                     ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(x.tmem + dcol, dadd64(d_rec, r * 32768 + r64::PART + ks * 256),
+                     dadd64(dx, ks * 256), id48, 1);
+    };
+    bool live = true;
+    for (int s = 0; s < x.n; ++s) {
+        const int r = s & 1;
+        gbar(BAR_BD, BAR_BD_THREADS);  // B_s written
+        if (leader && live) {
+            live = w64(ab, &sm.full[r], (uint32_t)(s >> 1) & 1u);
+            if (live) {
+                tc_fence_after();
+                tp_product(r, T_ACC2, d_b);
+                mma_commit(&sm.acc2_full);
+            }
+        }
+        __syncwarp();
+        gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s and D Delta_s written
+        if (leader && live) {
+            live = s < 1 || w64(ab, &sm.acc3_free, (uint32_t)(s - 1) & 1u);
+            if (live) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(x.tmem + T_ACC3, dadd64(d_kt, r * 32768 + ks * 2048),
+                             dadd64(d_dd, ks * 256), id_g3, ks > 0);
+                mma_commit(&sm.acc3_full);
+            }
+            // P Delta(s) after G1(s+1) (the next S step's product) was issued
+            live = live && (s + 1 >= x.n || w64(ab, &sm.g1_issued, (uint32_t)s & 1u)) &&
+                   (s < 1 || w64(ab, &sm.acc4_free, (uint32_t)(s - 1) & 1u));
+            if (live) {
+                tc_fence_after();
+                tp_product(r, T_ACC4, d_d);
+                mma_commit(&sm.acc4_full);
+                mma_commit(&sm.empty[r]);
+            }
+        }
+        __syncwarp();
+    }
+    if (leader) {
+        mma_commit(&sm.drain_d);
+        mbar_wait(&sm.drain_d, 0);
+    }
+    __syncwarp();
+}
+
+// ------------------------------------------------------------ S group (warps 0-7)
+__device__ void s64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
+                         const float* init_state, float* final_state) {
+    const int q = warp & 3, ch = warp >> 2;
+    const int k = 32 * q + lane;  // dk row
+    const int j0 = 24 * ch;
+    const uint32_t tl = x.tmem + lane_base64(warp);
+    constexpr uint32_t LO = NT * DK * 2;
+    const size_t srow = (((size_t)x.s * x.Hv + x.h) * DK + k) * DV + x.col0 + j0;
+    const int nvalid = DV - (x.col0 + j0);  // columns past dv are computed, never stored
+    int* ab = &sm.abort;
+    float Sm[24];
+#pragma unroll
+    for (int j = 0; j < 24; j += 4) {
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (init_state && j < nvalid) t = *reinterpret_cast<const float4*>(init_state + srow + j);
+        Sm[j] = t.x; Sm[j + 1] = t.y; Sm[j + 2] = t.z; Sm[j + 3] = t.w;
+    }
+    put24s(sm.s_op, LO, k, 3 * ch, DK, Sm, 1.f);
+    fence_async_smem();
+    gbar(BAR_S, BAR_S_THREADS);  // S_0 written
+    bool ok = true;
+    for (int s = 0; s < x.n; ++s) {
+        // the loads of block s landed (G1(s) was issued on them); this wait makes them visible
+        ok = ok && w64(ab, &sm.full[s & 1], (uint32_t)(s >> 1) & 1u);
+        const float gam = sm.vec[s & 1][r64::VEC_GAMMA];
+        ok = ok && w64(ab, &sm.acc3_full, (uint32_t)s & 1u);
+        if (ok) {
+            tc_fence_after();
+            ld_acc24s(tl + T_ACC3 + j0, gam, Sm);
+        }
+        warp_arrive64(&sm.acc3_free, lane);
+        if (s + 1 < x.n) {
+            // G1(s) read S_s from s_op: done before S_{s+1} replaces it
+            ok = ok && w64(ab, &sm.acc1_full[s & 1], (uint32_t)(s >> 1) & 1u);
+            if (ok) {
+                put24s(sm.s_op, LO, k, 3 * ch, DK, Sm, 1.f);
+                fence_async_smem();
+            }
+            gbar(BAR_S, BAR_S_THREADS);  // S_{s+1} written
+        }
+    }
+    if (ok && final_state && *(volatile int*)&sm.abort == 0) {
+#pragma unroll
+        for (int j = 0; j < 24; j += 4)
+            if (j < nvalid)
+                *reinterpret_cast<float4*>(final_state + srow + j) =
+                    make_float4(Sm[j], Sm[j + 1], Sm[j + 2], Sm[j + 3]);
+    }
+}
+
+// ---------------------------------------------------- BD group (warps 8, 9, 12, 13)
+__device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
+    const int q = warp & 3, ch = (warp - 8) >> 2;
+    const int r = 32 * q + lane;  // token of the block (accumulator rows 0-63)
+    const int j0 = 24 * ch;
+    const uint32_t tl = x.tmem + lane_base64(warp);
+    const int nv = DV - (x.col0 + j0);  // columns of V that exist
+    int* ab = &sm.abort;
+    bool live = true;
+    for (int s = 0; s < x.n; ++s) {
+        const int rs = s & 1;
+        live = live && w64(ab, &sm.full[rs], (uint32_t)(s >> 1) & 1u);
+        const float bet = sm.vec[rs][r64::VEC_BETA + r], wv = sm.vec[rs][r64::VEC_W + r];
+        const float d = sm.vec[rs][r64::VEC_D + r];
+        // V row r, columns j0 .. j0 + 23 of the tile: 16-byte chunks 3 ch + g of a
+        // 128-byte swizzled row (chunk c sits at c ^ (r % 8)); zero past the sequence or dv
+        const bool tok = x.t0 + (long long)s * C64 + r < x.t1;
+        uint4 vc[3];
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+            const int hf = r >> 5, rr = r & 31;
+            const int c = 3 * ch + g;
+            vc[g] = (tok && 8 * g < nv)
+                        ? *reinterpret_cast<const uint4*>(sm.vt[rs] + hf * 4096 + rr * 128 +
+                                                         ((c ^ (rr & 7)) << 4))
+                        : make_uint4(0, 0, 0, 0);
+        }
+        // B = beta V - w K S
+        live = live && w64(ab, &sm.acc1_full[s & 1], (uint32_t)(s >> 1) & 1u);
+        float v[24];
+#pragma unroll
+        for (int j = 0; j < 24; ++j) v[j] = 0.f;
+        if (live) {
+            tc_fence_after();
+            ld_acc24s(tl + T_ACC1 + 96 * (s & 1) + j0, 0.f, v);
+        }
+        warp_arrive64(&sm.acc1_free[s & 1], lane);
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+            const uint32_t wd[4] = {vc[g].x, vc[g].y, vc[g].z, vc[g].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[e]));
+                v[8 * g + 2 * e] = bet * fv.x - wv * v[8 * g + 2 * e];
+                v[8 * g + 2 * e + 1] = bet * fv.y - wv * v[8 * g + 2 * e + 1];
+            }
+        }
+        put24s(sm.b_op, OPB, r, 3 * ch, C64, v, 1.f);
+        fence_async_smem();
+        gbar(BAR_BD, BAR_BD_THREADS);  // B_s written: Delta(s)
+        // Delta = -acc2 rows 0-63; D Delta
+        live = live && w64(ab, &sm.acc2_full, (uint32_t)s & 1u);
+        if (live) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 24; ++j) v[j] = 0.f;
+            ld_acc24s(tl + T_ACC2 + j0, 0.f, v);
+            put24s(sm.d_op, OPB, r, 3 * ch, C64, v, -1.f);
+            put24s(sm.dd_op, OPB, r, 3 * ch, C64, v, -d);
+            fence_async_smem();
+        }
+        tc_fence_before();
+        gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s written: G3(s), P Delta(s)
+    }
+}
+
+// ---------------------------------------------- output group (warps 10, 11, 14, 15)
+__device__ void o64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
+                         float* __restrict__ out) {
+    const int q = warp & 3, ch = (warp - 8) >> 2;
+    const int i = 32 * (q - 2) + lane;  // token of the block (accumulator rows 64-127)
+    const int j0 = 24 * ch;
+    const uint32_t tl = x.tmem + lane_base64(warp);
+    const int nvalid = DV - (x.col0 + j0);
+    int* ab = &sm.abort;
+    float e_next = x.vec(0)[r64::VEC_E + i];
+    for (int s = 0; s < x.n; ++s) {
+        const float e = e_next;
+        if (s + 1 < x.n) e_next = x.vec(s + 1)[r64::VEC_E + i];
+        float o[24];
+#pragma unroll
+        for (int j = 0; j < 24; ++j) o[j] = 0.f;
+        if (!w64(ab, &sm.acc1_full[s & 1], (uint32_t)(s >> 1) & 1u)) break;
+        tc_fence_after();
+        ld_acc24s(tl + T_ACC1 + 96 * (s & 1) + j0, 0.f, o);
+        warp_arrive64(&sm.acc1_free[s & 1], lane);
+        if (!w64(ab, &sm.acc4_full, (uint32_t)s & 1u)) break;
+        tc_fence_after();
+        ld_acc24s(tl + T_ACC4 + j0, e, o);
+        warp_arrive64(&sm.acc4_free, lane);
+        const long long t = x.t0 + (long long)s * C64 + i;
+        float* st = &sm.o_st[i][j0];
+        bulk_wait_read_all();  // the previous block's copy of this segment has read it
+#pragma unroll
+        for (int j = 0; j < 24; j += 4)
+            *reinterpret_cast<float4*>(st + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
+        fence_async_smem();
+        if (t < x.t1 && nvalid > 0) {
+            bulk_store(out + ((size_t)t * x.Hv + x.h) * DV + x.col0 + j0, st,
+                       4u * (uint32_t)min(24, nvalid));
+            bulk_commit();
+        }
+    }
+    bulk_wait_all();
+}
+
+__global__ void __launch_bounds__(SP_THREADS, 1)
+state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v,
+               const uint8_t* __restrict__ ws,
+               const float* init_state, float* __restrict__ out, float* final_state,
+               const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    Sp64Smem& sm = *reinterpret_cast<Sp64Smem*>(smem_raw);
+    const int tile = blockIdx.x % NTILES;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    Sp64Ctx x;
+    x.h = (blockIdx.x / NTILES) % Hv;
+    x.s = blockIdx.x / (NTILES * Hv);
+    x.kh = x.h / (Hv / Hk);
+    x.Hv = Hv;
+    x.col0 = tile * NT;
+    seq_range(cu_seqlens, x.s, T, x.t0, x.t1);
+    x.n = (int)((x.t1 - x.t0 + C64 - 1) / C64);
+    x.rbase = r64::block_base(cu_seqlens, x.s, T);
+    x.ws = ws;
+    const int ncols = min(NT, DV - x.col0);
+    if (x.n == 0) {  // empty sequence: the final state is the initial one
+        if (final_state && tid < DK) {
+            const size_t row = (((size_t)x.s * Hv + x.h) * DK + tid) * DV + x.col0;
+            for (int j = 0; j < ncols; j += 4)
+                *reinterpret_cast<float4*>(final_state + row + j) =
+                    init_state ? *reinterpret_cast<const float4*>(init_state + row + j)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        return;
+    }
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (tid == 0) atomicExch(&g_tc64_status, 2);
+        return;
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], 2);      // G1 and the last P Delta product of the block
+            mbar_init(&sm.acc1_full[i], 1);
+            mbar_init(&sm.acc1_free[i], 8);  // BD and output warps
+        }
+        mbar_init(&sm.acc2_full, 1);
+        mbar_init(&sm.g1_issued, 1);
+        mbar_init(&sm.acc3_full, 1);
+        mbar_init(&sm.acc3_free, 8);  // S warps
+        mbar_init(&sm.acc4_full, 1);
+        mbar_init(&sm.acc4_free, 4);  // output warps
+        mbar_init(&sm.drain_s, 1);
+        mbar_init(&sm.drain_d, 1);
+        sm.abort = 0;
+        mbar_init_fence();
+        tma_prefetch_map(&tm_q);
+        tma_prefetch_map(&tm_k);
+        tma_prefetch_map(&tm_v);
+    }
+    if (warp == 0) tmem_alloc(&sm.tmem_base, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    x.tmem = sm.tmem_base;
+
+    if (warp < 8)
+        s64_role(sm, x, warp, lane, init_state, final_state);
+    else if (warp < 16)
+        ((warp & 3) < 2) ? bd_role(sm, x, warp, lane) : o64_role(sm, x, warp, lane, out);
+    else if (warp == 16)
+        load64_role(sm, x, lane, &tm_q, &tm_k, &tm_v);
+    else if (warp == 18)
+        d_issue_role(sm, x, lane);
+    else if (warp == 19)
+        g1_issue_role(sm, x, lane);
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(x.tmem, TMEM_COLS);
+    if (tid == 0 && sm.abort) atomicExch(&g_tc64_status, 1);
+}
+
+}  // namespace
+
+int read_and_clear_tc64_status() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc64_status, sizeof(int)) != cudaSuccess) return -1;
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_tc64_status, &zero, sizeof(int));
+    }
+    return v;
+}
+
+size_t prefill_tc64_workspace_bytes(const FwdParams& p) {
+    return (size_t)r64::max_records(p.cu_seqlens != nullptr, p.nseq, p.T) * p.Hv * r64::BYTES;
+}
+
+// The rule and its erase=False form with outputs (bf16, dk = dv = 128, chunk 32), on a
+// caller's workspace of at least prefill_tc64_workspace_bytes(p).
+cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t stream) {
+    if (p.in != InType::BF16 || p.dk != DK || p.dv != DV || p.chunk != 32 || p.v_zero ||
+        p.init_identity || !p.out)
+        return cudaErrorNotSupported;
+    const long long tokens = p.cu_seqlens ? (long long)p.T : (long long)p.nseq * p.T;
+    if (tokens <= 0 || tokens >= (1LL << 31) - 128) return cudaErrorNotSupported;
+    CUtensorMap mq, mk, mv;
+    if (!make_bf16_map(&mq, p.q, (uint64_t)p.Hk * DK, tokens) ||
+        !make_bf16_map(&mk, p.k, (uint64_t)p.Hk * DK, tokens) ||
+        !make_bf16_map(&mv, p.v, (uint64_t)p.Hv * DV, tokens))
+        return cudaErrorInvalidValue;
+    const long long nrec = r64::max_records(p.cu_seqlens != nullptr, p.nseq, p.T);
+    cudaError_t e = cudaFuncSetAttribute(intra64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(Prep64Smem));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(state64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(Sp64Smem));
+    if (e != cudaSuccess) return e;
+    intra64_kernel<<<(unsigned)(nrec * p.Hv), PREP64_THREADS, sizeof(Prep64Smem), stream>>>(
+        mq, mk, (const __nv_bfloat16*)p.a, (const __nv_bfloat16*)p.b, p.A_log, p.dt_bias,
+        p.cu_seqlens, p.T, p.nseq, p.Hk, p.Hv, p.erase, (uint8_t*)ws);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    state64_kernel<<<(unsigned)(p.nseq * p.Hv * NTILES), SP_THREADS, sizeof(Sp64Smem), stream>>>(
+        mq, mk, mv, (const uint8_t*)ws, p.init_state, p.out, p.final_state,
+        p.cu_seqlens, p.T, p.Hk, p.Hv);
+    return cudaGetLastError();
+}
+
+}  // namespace gdr
