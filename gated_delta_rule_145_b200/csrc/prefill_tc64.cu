@@ -115,6 +115,13 @@ __device__ __forceinline__ float scan32(float x, int lane) {
     return x;
 }
 
+// 2^x by the special-function unit (ex2.approx; results below the normal range flush to 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t lane_base64(int warp) { return (uint32_t)((warp & 3) * 32) << 16; }
 __device__ __forceinline__ uint64_t dadd64(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
@@ -152,25 +159,28 @@ __device__ __forceinline__ void store_chunk(uint8_t* hi, uint8_t* lo, uint32_t o
 struct alignas(1024) Prep64Smem {
     union {
         // per dk half (16 KB): K rows 0-63 | Q rows 64-127, 128-byte rows, 128-byte
-        // swizzle (two TMA boxes of 32 rows each).  Dead once the Gram product and the Q
-        // norms are done; A then takes the space.
+        // swizzle (two TMA boxes of 32 rows each).  Dead once the Gram product and the
+        // norms are done; the solve's arrays then take the space.
         uint8_t kq[2][16384];
-        float Am[C64][68];
+        struct {
+            float Am[C64][68];
+            float Tm[C64][68];  // T = (I + A)^-1, stored with its zero upper triangle
+            float Zm[32][36];   // coupling products
+        } w;
     };
-    float Tm[C64][68];  // T = (I + A)^-1, stored with its zero upper triangle
-    float Zm[32][36];   // coupling products
     alignas(16) float beta[C64];
     alignas(16) float G[C64];   // G of tokens 32-63 still lacks the first half's total
+    alignas(16) float G2[C64];  // the block's G times log2(e)
     alignas(16) float rk[C64];
     alignas(16) float rq[C64];
     uint64_t bar_tma, bar_mma;
     uint32_t tmem;
 };
-static_assert(sizeof(Prep64Smem) <= 57 * 1024, "four intra-block CTAs per SM");
+static_assert(sizeof(Prep64Smem) <= 44 * 1024, "five intra-block CTAs per SM");
 
 constexpr int PREP64_THREADS = 128;
 
-__global__ void __launch_bounds__(PREP64_THREADS, 4)
+__global__ void __launch_bounds__(PREP64_THREADS, 5)
 intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                const float* __restrict__ A_log, const float* __restrict__ dt_bias,
@@ -247,35 +257,27 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         __syncwarp();
     }
-    // ---- inverse norms of the Q rows (thread pair per row; the swizzle only permutes
-    //      16-byte pieces inside a row, which a sum ignores)
+    // ---- inverse norms of the K rows (0-63) and Q rows (64-127): a thread pair per row
+    //      (the swizzle only permutes 16-byte pieces inside a row, which a sum ignores)
+    if (tid < C64) sm.G2[tid] = (sm.G[tid] + (tid >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f;
     if (ok) {
-        const int row = tid >> 1, hf = tid & 1;
-        float ss = sumsq_line(sm.kq[hf] + 8192 + row * 128);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        if (hf == 0) sm.rq[row] = rsqrtf(ss + kNormEps) * rsqrtf((float)DK);
+#pragma unroll 1
+        for (int e = 0; e < 2; ++e) {
+            const int row = 64 * e + (tid >> 1), hf = tid & 1;
+            float ss = sumsq_line(sm.kq[hf] + row * 128);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            if (hf == 0) {
+                if (e == 0) sm.rk[row] = rsqrtf(ss + kNormEps);
+                else sm.rq[row - 64] = rsqrtf(ss + kNormEps) * rsqrtf((float)DK);
+            }
+        }
     }
     ok = __syncthreads_and(ok && mbar_wait(&sm.bar_mma, 0)) != 0;
     tc_fence_after();
-    // accumulator row 32 w + lane: warps 0, 1 rows of K K^T, warps 2, 3 rows of Q K^T
-    float v[C64];
-    if (ok) {
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-            tmem_ld16(tmem + lane_base64(warp) + 16 * q4, *reinterpret_cast<float(*)[16]>(&v[16 * q4]));
-        tmem_ld_wait();
-    }
-    if (warp < 2) {  // r_k from the diagonal of K K^T
-        const int i = 32 * warp + lane;
-        float dd = 0.f;
-#pragma unroll
-        for (int j = 0; j < C64; ++j) dd = j == i ? v[j] : dd;
-        sm.rk[i] = rsqrtf(dd + kNormEps);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 64);
     if (!ok) {
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tmem, 64);
         if (tid == 0) atomicExch(&g_tc64_status, 1);
         return;
     }
@@ -283,38 +285,52 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     auto Gf = [&](int j) { return sm.G[j] + (j >= 32 ? G31 : 0.f); };
 
     // ---- A rows into shared memory (warps 0, 1); P rows straight into the record's
-    //      image rows 64-127 (warps 2, 3)
-    if (warp < 2) {
-        const int i = 32 * warp + lane;
-        const float Gi = Gf(i), fa = erase ? sm.beta[i] * sm.rk[i] : 0.f;
-#pragma unroll
-        for (int j = 0; j < C64; j += 4) {
-            float4 o;
-            float* op = &o.x;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int jj = j + e;
-                const float av = fa * __expf(Gi - Gf(jj)) * sm.rk[jj] * v[jj];
-                op[e] = jj < i ? av : 0.f;
-            }
-            *reinterpret_cast<float4*>(&sm.Am[i][j]) = o;
-        }
-    } else {
-        const int i = 32 * (warp - 2) + lane;
-        const float Gi = Gf(i), fp = sm.rq[i];
-#pragma unroll
-        for (int kc = 0; kc < 8; ++kc) {
-            float p[8];
+    //      image rows 64-127 (warps 2, 3).  Accumulator row 32 w + lane (warps 0, 1: K K^T,
+    //      2, 3: Q K^T), read eight columns at a time.
+    {
+        const bool arow = warp < 2;
+        const int i = 32 * (warp & 1) + lane;
+        const float Gi2 = sm.G2[i];
+        const float f = arow ? (erase ? sm.beta[i] * sm.rk[i] : 0.f) : sm.rq[i];
+        // rows 0-31 (warps 0, 2) have nothing right of column 31: A there is never read and
+        // the image's P chunks are written as zeros below
+        const int kc_end = (warp & 1) ? 8 : 4;
+#pragma unroll 1
+        for (int kc = 0; kc < kc_end; ++kc) {
+            float v[8], p[8];
+            tmem_ld8(tmem + lane_base64(warp) + 8 * kc, v);
+            const float4 g0 = *reinterpret_cast<const float4*>(&sm.G2[8 * kc]);
+            const float4 g1 = *reinterpret_cast<const float4*>(&sm.G2[8 * kc + 4]);
+            const float4 r0 = *reinterpret_cast<const float4*>(&sm.rk[8 * kc]);
+            const float4 r1 = *reinterpret_cast<const float4*>(&sm.rk[8 * kc + 4]);
+            const float gj[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            const float rj[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int jj = 8 * kc + e;
-                const float pv = fp * __expf(Gi - Gf(jj)) * sm.rk[jj] * v[jj];
-                p[e] = jj <= i ? pv : 0.f;
+                const float pv = f * ex2_approx(Gi2 - gj[e]) * rj[e] * v[e];
+                p[e] = (jj < i || (!arow && jj == i)) ? pv : 0.f;
             }
-            store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(C64 + i, kc), p, 1.f);
+            if (arow) {
+                *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc]) = make_float4(p[0], p[1], p[2], p[3]);
+                *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc + 4]) = make_float4(p[4], p[5], p[6], p[7]);
+            } else {
+                store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(C64 + i, kc), p, 1.f);
+            }
+        }
+        if (!arow && kc_end == 4) {
+#pragma unroll
+            for (int kc = 4; kc < 8; ++kc) {
+                const uint32_t off = r64::k_off(C64 + i, kc);
+                *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
+            }
         }
     }
+    tc_fence_before();
     __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
 
     // ---- T = (I + A)^-1.  The four diagonal 16 x 16 blocks by forward substitution, one
     //      column per lane (warps 0 and 1: lanes 0-15 and 16-31 take one block each);
@@ -327,23 +343,22 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             float s0 = i == j ? 1.f : 0.f, s1 = 0.f;
 #pragma unroll
             for (int m = 0; m < (i & ~1); m += 2) {
-                const float2 av = *reinterpret_cast<const float2*>(&sm.Am[o + i][o + m]);
+                const float2 av = *reinterpret_cast<const float2*>(&sm.w.Am[o + i][o + m]);
                 s0 -= av.x * x[m];
                 s1 -= av.y * x[m + 1];
             }
-            if (i & 1) s0 -= sm.Am[o + i][o + i - 1] * x[i - 1];
+            if (i & 1) s0 -= sm.w.Am[o + i][o + i - 1] * x[i - 1];
             x[i] = s0 + s1;
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sm.Tm[o + i][o + j] = x[i];
+        for (int i = 0; i < 16; ++i) sm.w.Tm[o + i][o + j] = x[i];
     } else {
-        // rows 16 bi .. 16 bi + 15, columns right of the diagonal block: 6 blocks
-        for (int e = tid - 64; e < 6 * 256; e += 64) {
+        // the zero blocks above the diagonal inside each 32-token block, (0,1) and (2,3),
+        // which the 32-level coupling reads (the upper-right 32 x 32 block of the image is
+        // written as zeros directly)
+        for (int e = tid - 64; e < 2 * 256; e += 64) {
             const int blk = e >> 8, w = e & 255, r = w >> 4, cc = w & 15;
-            // blocks (row band, column band): (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-            const int rb = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-            const int cb = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            sm.Tm[16 * rb + r][16 * cb + cc] = 0.f;
+            sm.w.Tm[32 * blk + r][32 * blk + 16 + cc] = 0.f;
         }
     }
     __syncthreads();
@@ -354,11 +369,11 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
-            const float a_ = sm.Am[o + 16 + i][o + m];
-            const float4 t4 = *reinterpret_cast<const float4*>(&sm.Tm[o + m][o + jc]);
+            const float a_ = sm.w.Am[o + 16 + i][o + m];
+            const float4 t4 = *reinterpret_cast<const float4*>(&sm.w.Tm[o + m][o + jc]);
             z[0] += a_ * t4.x; z[1] += a_ * t4.y; z[2] += a_ * t4.z; z[3] += a_ * t4.w;
         }
-        *reinterpret_cast<float4*>(&sm.Zm[16 * bi + i][jc]) = make_float4(z[0], z[1], z[2], z[3]);
+        *reinterpret_cast<float4*>(&sm.w.Zm[16 * bi + i][jc]) = make_float4(z[0], z[1], z[2], z[3]);
     }
     __syncthreads();
     {
@@ -368,11 +383,11 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float t[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
-            const float tv = sm.Tm[o + 16 + i][o + 16 + m];
-            const float4 z4 = *reinterpret_cast<const float4*>(&sm.Zm[16 * bi + m][jc]);
+            const float tv = sm.w.Tm[o + 16 + i][o + 16 + m];
+            const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Zm[16 * bi + m][jc]);
             t[0] += tv * z4.x; t[1] += tv * z4.y; t[2] += tv * z4.z; t[3] += tv * z4.w;
         }
-        *reinterpret_cast<float4*>(&sm.Tm[o + 16 + i][o + jc]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+        *reinterpret_cast<float4*>(&sm.w.Tm[o + 16 + i][o + jc]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
     }
     __syncthreads();
     {
@@ -384,14 +399,14 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int q = 0; q < 8; ++q) z[q] = 0.f;
 #pragma unroll 4
         for (int m = 0; m < 32; ++m) {
-            const float a_ = sm.Am[32 + i][m];
-            const float4 t0v = *reinterpret_cast<const float4*>(&sm.Tm[m][j0]);
-            const float4 t1v = *reinterpret_cast<const float4*>(&sm.Tm[m][j0 + 4]);
+            const float a_ = sm.w.Am[32 + i][m];
+            const float4 t0v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0]);
+            const float4 t1v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0 + 4]);
             z[0] += a_ * t0v.x; z[1] += a_ * t0v.y; z[2] += a_ * t0v.z; z[3] += a_ * t0v.w;
             z[4] += a_ * t1v.x; z[5] += a_ * t1v.y; z[6] += a_ * t1v.z; z[7] += a_ * t1v.w;
         }
-        *reinterpret_cast<float4*>(&sm.Zm[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
-        *reinterpret_cast<float4*>(&sm.Zm[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
+        *reinterpret_cast<float4*>(&sm.w.Zm[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
+        *reinterpret_cast<float4*>(&sm.w.Zm[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
     }
     __syncthreads();
     {
@@ -402,22 +417,29 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int q = 0; q < 8; ++q) t[q] = 0.f;
 #pragma unroll 4
         for (int m = 0; m < 32; ++m) {
-            const float tv = sm.Tm[32 + i][32 + m];
-            const float4 z0 = *reinterpret_cast<const float4*>(&sm.Zm[m][j0]);
-            const float4 z1 = *reinterpret_cast<const float4*>(&sm.Zm[m][j0 + 4]);
+            const float tv = sm.w.Tm[32 + i][32 + m];
+            const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Zm[m][j0]);
+            const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Zm[m][j0 + 4]);
             t[0] += tv * z0.x; t[1] += tv * z0.y; t[2] += tv * z0.z; t[3] += tv * z0.w;
             t[4] += tv * z1.x; t[5] += tv * z1.y; t[6] += tv * z1.z; t[7] += tv * z1.w;
         }
-        *reinterpret_cast<float4*>(&sm.Tm[32 + i][j0]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
-        *reinterpret_cast<float4*>(&sm.Tm[32 + i][j0 + 4]) = make_float4(-t[4], -t[5], -t[6], -t[7]);
+        *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+        *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0 + 4]) = make_float4(-t[4], -t[5], -t[6], -t[7]);
     }
     __syncthreads();
-    // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread)
+    // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread); rows 0-31 x
+    //      columns 32-63 are zero
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         const int task = tid + PREP64_THREADS * e, row = task >> 3, kc = task & 7;
-        store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(row, kc),
-                    &sm.Tm[row][8 * kc], -1.f);
+        if (row < 32 && kc >= 4) {
+            const uint32_t off = r64::k_off(row, kc);
+            *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
+        } else {
+            store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(row, kc),
+                        &sm.w.Tm[row][8 * kc], -1.f);
+        }
     }
     // ---- vectors
     if (tid < C64) {
@@ -529,17 +551,17 @@ __device__ __forceinline__ void put24s(uint8_t* op, uint32_t lo_off, int k, int 
     }
 }
 
-// v = sc * v + (hi + lo halves of a [hi | lo] accumulator), 24 columns from taddr.
+// v = (sc * v + hi) + lo over 24 columns of a [hi | lo] accumulator from taddr (all four
+// loads in flight before one wait).
 __device__ __forceinline__ void ld_acc24s(uint32_t taddr, float sc, float (&v)[24]) {
+    float hi[24], lo[24];
+    tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&hi[0]));
+    tmem_ld8(taddr + 16, &hi[16]);
+    tmem_ld16(taddr + NT, *reinterpret_cast<float(*)[16]>(&lo[0]));
+    tmem_ld8(taddr + NT + 16, &lo[16]);
+    tmem_ld_wait();
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
-        float t[24];
-        tmem_ld16(taddr + NT * part, *reinterpret_cast<float(*)[16]>(&t[0]));
-        tmem_ld8(taddr + NT * part + 16, &t[16]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 24; ++i) v[i] = (part == 0 ? sc * v[i] : v[i]) + t[i];
-    }
+    for (int i = 0; i < 24; ++i) v[i] = (sc * v[i] + hi[i]) + lo[i];
 }
 
 struct Sp64Ctx {
@@ -601,11 +623,13 @@ __device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
     bool live = true;
     for (int s = 0; s < x.n; ++s) {
         const int r = s & 1, x1 = s & 1;
-        gbar(BAR_S, BAR_S_THREADS);  // S_s written
-        if (leader && live) {
+        // what G1(s) needs besides S_s, waited for before S_s is
+        if (leader && live)
             live = w64(ab, &sm.full[r], (uint32_t)(s >> 1) & 1u) &&        // tiles of s
                    (s < 2 || w64(ab, &sm.acc1_free[x1], (uint32_t)((s >> 1) - 1) & 1u));
-            if (live) {
+        gbar(BAR_S, BAR_S_THREADS);  // S_s written
+        if (leader && live) {
+            {
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
@@ -653,20 +677,18 @@ __device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
     bool live = true;
     for (int s = 0; s < x.n; ++s) {
         const int r = s & 1;
+        if (leader && live) live = w64(ab, &sm.full[r], (uint32_t)(s >> 1) & 1u);
         gbar(BAR_BD, BAR_BD_THREADS);  // B_s written
         if (leader && live) {
-            live = w64(ab, &sm.full[r], (uint32_t)(s >> 1) & 1u);
-            if (live) {
-                tc_fence_after();
-                tp_product(r, T_ACC2, d_b);
-                mma_commit(&sm.acc2_full);
-            }
+            tc_fence_after();
+            tp_product(r, T_ACC2, d_b);
+            mma_commit(&sm.acc2_full);
         }
         __syncwarp();
+        if (leader && live) live = s < 1 || w64(ab, &sm.acc3_free, (uint32_t)(s - 1) & 1u);
         gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s and D Delta_s written
         if (leader && live) {
-            live = s < 1 || w64(ab, &sm.acc3_free, (uint32_t)(s - 1) & 1u);
-            if (live) {
+            {
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
