@@ -481,8 +481,9 @@ constexpr int O_PITCH = 52;             // floats: 208 B rows, 16-byte aligned
 // The S and BD groups read nothing from global memory inside the loop: a named barrier
 // orders memory like membar.cta and so waits for a warp's global loads still in flight.
 //   18             issues Delta, K^T D Delta and P Delta (meets the BD group on BAR_BD);
-//                  P Delta(s) only after G1(s+1) was issued, so that the tensor pipe runs
-//                  the chain's product first
+//                  P Delta(s) right behind K^T D Delta(s), so that it runs while the S group
+//                  forms the next state (from another warp, or after G1(s+1), it held up the
+//                  chain's products on the tensor pipe)
 //   19             issues [K; Q] [S hi | lo] (meets the S group on BAR_S)
 //   17             no role
 struct alignas(1024) Sp64Smem {
@@ -497,7 +498,7 @@ struct alignas(1024) Sp64Smem {
     uint8_t dd_op[2 * OPB];         // diag(D) Delta
     float o_st[C64][O_PITCH];       // output rows of block s (pitch: conflict-free v4 stores)
     uint64_t full[2], empty[2];
-    uint64_t acc1_full[2], acc1_free[2], acc2_full, g1_issued;
+    uint64_t acc1_full[2], acc1_free[2], acc2_full;
     uint64_t acc3_full, acc3_free, acc4_full, acc4_free, drain_s, drain_d;
     uint32_t tmem_base;
     int abort;
@@ -638,7 +639,6 @@ __device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
                              dadd64(d_s, ks * 256), id96, ks > 0);
                 mma_commit(&sm.acc1_full[x1]);
                 mma_commit(&sm.empty[r]);
-                if (s >= 1) mbar_arrive(&sm.g1_issued);
             }
         }
         __syncwarp();
@@ -696,9 +696,8 @@ __device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
                              dadd64(d_dd, ks * 256), id_g3, ks > 0);
                 mma_commit(&sm.acc3_full);
             }
-            // P Delta(s) after G1(s+1) (the next S step's product) was issued
-            live = live && (s + 1 >= x.n || w64(ab, &sm.g1_issued, (uint32_t)s & 1u)) &&
-                   (s < 1 || w64(ab, &sm.acc4_free, (uint32_t)(s - 1) & 1u));
+            // P Delta(s) right behind G3(s): it runs while the S group forms S_{s+1}
+            live = live && (s < 1 || w64(ab, &sm.acc4_free, (uint32_t)(s - 1) & 1u));
             if (live) {
                 tc_fence_after();
                 tp_product(r, T_ACC4, d_d);
@@ -915,7 +914,6 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&sm.acc1_free[i], 8);  // BD and output warps
         }
         mbar_init(&sm.acc2_full, 1);
-        mbar_init(&sm.g1_issued, 1);
         mbar_init(&sm.acc3_full, 1);
         mbar_init(&sm.acc3_free, 8);  // S warps
         mbar_init(&sm.acc4_full, 1);
