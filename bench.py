@@ -616,7 +616,7 @@ def run_ours(args, dist):
                 "roofline": {
                     "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                    "traffic": recorded_traffic("prefill_tc.cu"), "peak_source": pk["source"],
+                    "traffic": recorded_traffic("prefill_tc64.cu"), "peak_source": pk["source"],
                     "alg_bytes_per_launch": alg_b, "alg_flops_per_launch": alg_f,
                     "kernel_ms": round(pre["kernel_ms"], 4),
                     "kernel_ms_median": round(pre["kernel_ms_median"], 4),

@@ -125,12 +125,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ uint32_t lane_base64(int warp) { return (uint32_t)((warp & 3) * 32) << 16; }
 __device__ __forceinline__ uint64_t dadd64(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
-// Sum of squares of the 64 bf16 values in 128 bytes of shared memory.
-__device__ __forceinline__ float sumsq_line(const uint8_t* line) {
+// Sum of squares of the 64 bf16 values in 128 bytes of shared memory; the 16-byte pieces
+// are visited from piece `rot` on, so that lanes on different rows read different banks.
+__device__ __forceinline__ float sumsq_line(const uint8_t* line, int rot) {
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const uint4 u = *reinterpret_cast<const uint4*>(line + 16 * j);
+        const uint4 u = *reinterpret_cast<const uint4*>(line + 16 * ((j + rot) & 7));
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -264,7 +265,7 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll 1
         for (int e = 0; e < 2; ++e) {
             const int row = 64 * e + (tid >> 1), hf = tid & 1;
-            float ss = sumsq_line(sm.kq[hf] + row * 128);
+            float ss = sumsq_line(sm.kq[hf] + row * 128, row + 4 * hf);
             ss += __shfl_xor_sync(0xffffffffu, ss, 1);
             if (hf == 0) {
                 if (e == 0) sm.rk[row] = rsqrtf(ss + kNormEps);
@@ -428,10 +429,12 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     __syncthreads();
     // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread); rows 0-31 x
-    //      columns 32-63 are zero
+    //      columns 32-63 are zero.  Eight consecutive lanes take the eight rows of one
+    //      8-row group at one chunk: one 128-byte line of the image.
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const int task = tid + PREP64_THREADS * e, row = task >> 3, kc = task & 7;
+        const int task = tid + PREP64_THREADS * e;
+        const int row = 8 * (task >> 6) + (task & 7), kc = (task >> 3) & 7;
         if (row < 32 && kc >= 4) {
             const uint32_t off = r64::k_off(row, kc);
             *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);

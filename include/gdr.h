@@ -37,7 +37,7 @@
  *     error taken from cudaGetLastError (which clears it).
  *   - Supported head sizes: dk == dv in {32, 64, 128}; chunk == 32.
  *   - Memory: the bf16 chunked prefill at dk = dv = 128 needs a workspace of
- *     16896 bytes per (chunk, value head) -- 208 MB for T = 8192, Hv = 48 -- which the
+ *     33808 bytes per (64-token block, value head) -- 208 MB for T = 8192, Hv = 48 -- which the
  *     library takes, per call, from a private stream-ordered pool of the current device
  *     (cudaMallocFromPoolAsync on `stream`, returned with cudaFreeAsync on the same
  *     stream once the call's kernels are enqueued).  Freed memory stays cached in the pool
@@ -108,9 +108,9 @@ GDR_API int gdr_prefill_chunked(const void* q, const void* k, const void* v, con
  * with dk = dv = 128, chunk = 32 and T >= 1 (anything else returns GDR_ERR_UNSUPPORTED;
  * use gdr_prefill_chunked there).  Instead of a pooled workspace the call uses a fixed
  * 64 MiB scratch array compiled into the library, which every device that loads the
- * library holds until the process exits.  The workspace needed is 16896 bytes per
- * (chunk, value head) -- dense mode B * ceil(T / 32) * Hv records, varlen mode at most
- * ((T + 31 B) / 32 + 1) * Hv -- so at most 3971 records fit (e.g. T = 2560 at Hv = 48);
+ * library holds until the process exits.  The workspace needed is 33808 bytes per
+ * (64-token block, value head) -- dense mode B * ceil(T / 64) * Hv records, varlen mode at
+ * most ((T + 63 B) / 64 + 1) * Hv -- so at most 1984 records fit (e.g. T = 2624 at Hv = 48);
  * larger calls return GDR_ERR_TOO_LARGE before anything is enqueued.  It calls no
  * allocator (no cudaMalloc, cudaMallocAsync or cudaFree).
  *   - The first call on a device looks up the scratch array's device address

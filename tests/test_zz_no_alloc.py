@@ -33,8 +33,10 @@ def _fake(**kw):
 
 
 def test_noalloc_refuses_what_does_not_fit():
-    # 128 chunks x 48 heads = 6144 records of 16896 bytes > 64 MiB
+    # 64 blocks of 64 tokens x 48 heads = 3072 records of 33808 bytes > 64 MiB
     assert _fake(T=4096, Hk=48, Hv=48) == gdr.GDR_ERR_TOO_LARGE
+    # just past the limit: 42 blocks x 48 heads = 2016 records > 1984 = 64 MiB / 33808
+    assert _fake(T=2625, Hk=48, Hv=48) == gdr.GDR_ERR_TOO_LARGE
     # the tensor-core variant only: other head sizes, chunk sizes or empty inputs are
     # left to gdr_prefill_chunked
     assert _fake(dk=64, dv=64) == gdr.GDR_ERR_UNSUPPORTED
