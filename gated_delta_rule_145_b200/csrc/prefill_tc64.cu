@@ -316,6 +316,12 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (arow) {
                 *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc]) = make_float4(p[0], p[1], p[2], p[3]);
                 *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc + 4]) = make_float4(p[4], p[5], p[6], p[7]);
+                // A_ba (rows 32-63, columns 0-31) also transposed into the unused top-right
+                // quarter of Am: Am[j][32 + i'] = A[32 + i'][j]
+                if (warp == 1 && kc < 4) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) sm.w.Am[8 * kc + e][32 + lane] = p[e];
+                }
             } else {
                 store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(C64 + i, kc), p, 1.f);
             }
@@ -378,12 +384,14 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     __syncthreads();
     {
-        // T[b+16.., b..] = -T[b+16.., b+16..] Z (the lower diagonal block has its zero
-        // upper triangle stored, so all 16 terms are summed)
+        // T[b+16.., b..] = -T[b+16.., b+16..] Z.  That block is lower triangular: row i needs
+        // m <= i only; a warp's rows end at 7 or 15, and the zero upper triangle it still
+        // reads below that is stored.
         const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
+        const int mend = (warp & 1) ? 16 : 8;
         float t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
+#pragma unroll 8
+        for (int m = 0; m < mend; ++m) {
             const float tv = sm.w.Tm[o + 16 + i][o + 16 + m];
             const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Zm[16 * bi + m][jc]);
             t[0] += tv * z4.x; t[1] += tv * z4.y; t[2] += tv * z4.z; t[3] += tv * z4.w;
@@ -392,15 +400,17 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     __syncthreads();
     {
-        // 32-level coupling: Z = A_ba T_a (rows 32-63, columns 0-31), thread -> row i,
-        // columns 8 cg .. 8 cg + 7
-        const int i = tid >> 2, j0 = 8 * (tid & 3);
+        // 32-level coupling: Z = A_ba T_a (rows 32-63, columns 0-31), warp w -> columns
+        // 8 w .. 8 w + 7, lane -> row.  T_a is lower triangular: column j needs m >= j, so
+        // the warp starts at m = 8 w (the zeros it reads above the diagonal are stored);
+        // A_ba comes from its transposed copy (consecutive lanes, consecutive words).
+        const int i = lane, j0 = 8 * warp;
         float z[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) z[q] = 0.f;
 #pragma unroll 4
-        for (int m = 0; m < 32; ++m) {
-            const float a_ = sm.w.Am[32 + i][m];
+        for (int m = j0; m < 32; ++m) {
+            const float a_ = sm.w.Am[m][32 + i];
             const float4 t0v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0]);
             const float4 t1v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0 + 4]);
             z[0] += a_ * t0v.x; z[1] += a_ * t0v.y; z[2] += a_ * t0v.z; z[3] += a_ * t0v.w;
@@ -411,13 +421,14 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     __syncthreads();
     {
-        // T_ba = -T_b Z
+        // T_ba = -T_b Z.  T_b is lower triangular: row i needs m <= i only; warp w holds rows
+        // 8 w .. 8 w + 7 (the zero upper triangle it reads below 8 w + 8 is stored).
         const int i = tid >> 2, j0 = 8 * (tid & 3);
         float t[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) t[q] = 0.f;
 #pragma unroll 4
-        for (int m = 0; m < 32; ++m) {
+        for (int m = 0; m < 8 * warp + 8; ++m) {
             const float tv = sm.w.Tm[32 + i][32 + m];
             const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Zm[m][j0]);
             const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Zm[m][j0 + 4]);
