@@ -481,25 +481,25 @@ constexpr uint32_t T_ACC4 = 384;  // 96: rows 64-127 P Delta
 constexpr uint32_t OPB = NT * C64 * 2;  // one K = 64 x N = 48 bf16 operand part (6144 B)
 constexpr int O_PITCH = 52;             // floats: 208 B rows, 16-byte aligned
 
-// Warp roles
+// Warp roles (a step's latency is mostly the per-thread length of its epilogues: the BD
+// group's two run on six warps; twelve S warps at 768 threads ran slower than eight)
 //   0-7            S group: the state slice in registers (row 32 (w % 4) + lane, 24 columns
 //                  per warp half); S <- gamma S + K^T D Delta and the state's hi/lo operand
-//   8, 9, 12, 13   BD group (accumulator rows 0-63): B = diag(beta) V - diag(w) K S and
-//                  Delta, D Delta
+//   8, 9, 12, 13,  BD group (accumulator rows 0-63, 16 columns per warp): B = diag(beta) V -
+//   16, 17         diag(w) K S and Delta, D Delta
 //   10, 11, 14, 15 output group (accumulator rows 64-127): O = E Q S + P Delta, staged in
 //                  shared memory and written by one bulk copy per row segment (per-lane
 //                  stores to rows 24 KB apart would hold up the memory pipe that the
 //                  operand stores of the chain use)
-//   16             loads: TMA tiles [K; Q] and V, the record image [-T; P] and its
-//                  vectors, two-deep ring
 // The S and BD groups read nothing from global memory inside the loop: a named barrier
 // orders memory like membar.cta and so waits for a warp's global loads still in flight.
 //   18             issues Delta, K^T D Delta and P Delta (meets the BD group on BAR_BD);
 //                  P Delta(s) right behind K^T D Delta(s), so that it runs while the S group
 //                  forms the next state (from another warp, or after G1(s+1), it held up the
 //                  chain's products on the tensor pipe)
-//   19             issues [K; Q] [S hi | lo] (meets the S group on BAR_S)
-//   17             no role
+//   19             issues [K; Q] [S hi | lo] (meets the S group on BAR_S) and the loads:
+//                  TMA tiles [K; Q] and V, the record image [-T; P] and its vectors,
+//                  two-deep ring
 struct alignas(1024) Sp64Smem {
     uint8_t kq[2][32768];   // block s: per dk half (16 KB) K rows 0-63 | Q rows 64-127
     uint8_t rec[2][32768];  // block s: [-T; P] hi (16 KB), lo (16 KB)
@@ -532,7 +532,7 @@ __device__ __forceinline__ bool w64(int* abort, uint64_t* bar, uint32_t parity) 
 // warp.  Every warp of a pair runs every barrier of it, also once the kernel is aborting
 // (its waits then return at once), so a timed-out wait cannot strand a barrier.
 constexpr uint32_t BAR_S = 1, BAR_BD = 2;
-constexpr uint32_t BAR_S_THREADS = 9 * 32, BAR_BD_THREADS = 5 * 32;
+constexpr uint32_t BAR_S_THREADS = 9 * 32, BAR_BD_THREADS = 7 * 32;
 
 __device__ __forceinline__ void gbar(uint32_t id, uint32_t nthreads) {
     __syncwarp();
@@ -566,6 +566,34 @@ __device__ __forceinline__ void put24s(uint8_t* op, uint32_t lo_off, int k, int 
     }
 }
 
+// 16 fp32 values (times sc) of K-row k (column groups g0, g0 + 1) as the hi and lo parts
+// of an MN-major operand whose lo part starts lo_off bytes after the hi part.
+__device__ __forceinline__ void put16s(uint8_t* op, uint32_t lo_off, int k, int g0, int krows,
+                                       const float (&v)[16], float sc) {
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        uint4 hv, lv;
+        split2(sc * v[8 * g + 0], sc * v[8 * g + 1], hv.x, lv.x);
+        split2(sc * v[8 * g + 2], sc * v[8 * g + 3], hv.y, lv.y);
+        split2(sc * v[8 * g + 4], sc * v[8 * g + 5], hv.z, lv.z);
+        split2(sc * v[8 * g + 6], sc * v[8 * g + 7], hv.w, lv.w);
+        const uint32_t o = mn_off64(k, g0 + g, krows);
+        *reinterpret_cast<uint4*>(op + o) = hv;
+        *reinterpret_cast<uint4*>(op + lo_off + o) = lv;
+    }
+}
+
+// v = (sc * v + hi) + lo over 16 columns of a [hi | lo] accumulator from taddr (both
+// loads in flight before one wait).
+__device__ __forceinline__ void ld_acc16s(uint32_t taddr, float sc, float (&v)[16]) {
+    float hi[16], lo[16];
+    tmem_ld16(taddr, hi);
+    tmem_ld16(taddr + NT, lo);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = (sc * v[i] + hi[i]) + lo[i];
+}
+
 // v = (sc * v + hi) + lo over 24 columns of a [hi | lo] accumulator from taddr (all four
 // loads in flight before one wait).
 __device__ __forceinline__ void ld_acc24s(uint32_t taddr, float sc, float (&v)[24]) {
@@ -593,49 +621,46 @@ struct Sp64Ctx {
     }
 };
 
-// ------------------------------------------------------------------- loads (warp 16)
-__device__ void load64_role(Sp64Smem& sm, const Sp64Ctx& x, int lane, const CUtensorMap* tm_q,
+// ------------------------------------------------------------------- loads
+// Block s's TMA tiles [K; Q] and V, its record image [-T; P] and vectors into ring slot
+// s & 1, counted on full[s & 1] (one thread).
+__device__ void issue_loads(Sp64Smem& sm, const Sp64Ctx& x, int s, const CUtensorMap* tm_q,
                             const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
-    int armed = -1;
-    for (int s = 0; s < x.n; ++s) {
-        const int r = s & 1, use = s >> 1;
-        if (use > 0 && !w64(&sm.abort, &sm.empty[r], (uint32_t)(use - 1) & 1u)) break;
-        if (lane == 0) {
-            uint64_t* bar = &sm.full[r];
-            mbar_arrive_expect_tx(bar, 10u * 4096u + 2u * r64::PART + r64::VEC_BYTES);
-            const int y = (int)(x.t0 + (long long)s * C64);
-            for (int hf = 0; hf < 2; ++hf) {
-                const int xx = x.kh * DK + 64 * hf;
-                uint8_t* base = sm.kq[r] + 16384 * hf;
-                tma_load_2d(base, tm_k, xx, y, bar);
-                tma_load_2d(base + 4096, tm_k, xx, y + 32, bar);
-                tma_load_2d(base + 8192, tm_q, xx, y, bar);
-                tma_load_2d(base + 12288, tm_q, xx, y + 32, bar);
-            }
-            tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, y, bar);
-            tma_load_2d(sm.vt[r] + 4096, tm_v, x.h * DV + x.col0, y + 32, bar);
-            const uint8_t* rc = x.record(s);
-            bulk_load(sm.rec[r], rc + r64::OFF_A, r64::PART, bar);
-            bulk_load(sm.rec[r] + r64::PART, rc + r64::OFF_A + r64::PART, r64::PART, bar);
-            bulk_load(sm.vec[r], rc + r64::OFF_VEC, r64::VEC_BYTES, bar);
-        }
-        __syncwarp();
-        armed = s;
+    const int r = s & 1;
+    uint64_t* bar = &sm.full[r];
+    mbar_arrive_expect_tx(bar, 10u * 4096u + 2u * r64::PART + r64::VEC_BYTES);
+    const int y = (int)(x.t0 + (long long)s * C64);
+#pragma unroll 1
+    for (int hf = 0; hf < 2; ++hf) {
+        const int xx = x.kh * DK + 64 * hf;
+        uint8_t* base = sm.kq[r] + 16384 * hf;
+        tma_load_2d(base, tm_k, xx, y, bar);
+        tma_load_2d(base + 4096, tm_k, xx, y + 32, bar);
+        tma_load_2d(base + 8192, tm_q, xx, y, bar);
+        tma_load_2d(base + 12288, tm_q, xx, y + 32, bar);
     }
-    // every copy this warp started has landed before the CTA may exit
-    for (int s = max(0, armed - 1); s <= armed; ++s) mbar_wait(&sm.full[s & 1], (uint32_t)(s >> 1) & 1u);
-    __syncwarp();
+    tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, y, bar);
+    tma_load_2d(sm.vt[r] + 4096, tm_v, x.h * DV + x.col0, y + 32, bar);
+    const uint8_t* rc = x.record(s);
+    bulk_load(sm.rec[r], rc + r64::OFF_A, r64::PART, bar);
+    bulk_load(sm.rec[r] + r64::PART, rc + r64::OFF_A + r64::PART, r64::PART, bar);
+    bulk_load(sm.vec[r], rc + r64::OFF_VEC, r64::VEC_BYTES, bar);
 }
 
-// ---------------------------------------------------------- issuing warps (18, 19)
-// Warp 19: G1(s) = [K_s; Q_s] [S_s hi | lo] into acc1[s & 1].
-__device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
+// Warp 19: G1(s) = [K_s; Q_s] [S_s hi | lo] into acc1[s & 1]; also the loads, a block
+// ahead: after G1(s), block s + 1 into the slot that block s - 1 has freed.
+__device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane, const CUtensorMap* tm_q,
+                              const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
     const uint32_t id96 = idesc_bf16(128, 2 * NT, 0, 1);
     const uint64_t d_kq = sdesc(smem_u32(sm.kq[0]), 16, 1024, kSw128);  // [K;Q] K-major
     const uint64_t d_s = sdesc(smem_u32(sm.s_op), 128, 2048, kSwNone);
     const bool leader = lane == 0;
     int* ab = &sm.abort;
     bool live = true;
+    int armed = min(x.n, 2) - 1;  // the last block whose loads were issued
+    if (leader)
+        for (int s = 0; s <= armed; ++s) issue_loads(sm, x, s, tm_q, tm_k, tm_v);
+    __syncwarp();
     for (int s = 0; s < x.n; ++s) {
         const int r = s & 1, x1 = s & 1;
         // what G1(s) needs besides S_s, waited for before S_s is
@@ -654,12 +679,23 @@ __device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
                 mma_commit(&sm.acc1_full[x1]);
                 mma_commit(&sm.empty[r]);
             }
+            // block s + 1 into slot (s + 1) & 1, once block s - 1 is done with it
+            if (live && s >= 1 && s + 1 < x.n) {
+                live = w64(ab, &sm.empty[(s + 1) & 1], (uint32_t)((s - 1) >> 1) & 1u);
+                if (live) {
+                    issue_loads(sm, x, s + 1, tm_q, tm_k, tm_v);
+                    armed = s + 1;
+                }
+            }
         }
         __syncwarp();
     }
     if (leader) {
         mma_commit(&sm.drain_s);
         mbar_wait(&sm.drain_s, 0);
+        // every copy this warp started has landed before the CTA may exit
+        for (int s = max(0, armed - 1); s <= armed; ++s)
+            mbar_wait(&sm.full[s & 1], (uint32_t)(s >> 1) & 1u);
     }
     __syncwarp();
 }
@@ -779,11 +815,13 @@ __device__ void s64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
     }
 }
 
-// ---------------------------------------------------- BD group (warps 8, 9, 12, 13)
+// ---------------------------------------- BD group (warps 8, 9, 12, 13, 16, 17)
+// Warp w: accumulator rows 32 (w % 4) + lane (tokens 0-63), columns 16 ct .. 16 ct + 15 with
+// ct = (w - 8) / 4.
 __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
-    const int q = warp & 3, ch = (warp - 8) >> 2;
+    const int q = warp & 3, ct = (warp - 8) >> 2;
     const int r = 32 * q + lane;  // token of the block (accumulator rows 0-63)
-    const int j0 = 24 * ch;
+    const int j0 = 16 * ct;
     const uint32_t tl = x.tmem + lane_base64(warp);
     const int nv = DV - (x.col0 + j0);  // columns of V that exist
     int* ab = &sm.abort;
@@ -793,14 +831,14 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
         live = live && w64(ab, &sm.full[rs], (uint32_t)(s >> 1) & 1u);
         const float bet = sm.vec[rs][r64::VEC_BETA + r], wv = sm.vec[rs][r64::VEC_W + r];
         const float d = sm.vec[rs][r64::VEC_D + r];
-        // V row r, columns j0 .. j0 + 23 of the tile: 16-byte chunks 3 ch + g of a
+        // V row r, columns j0 .. j0 + 15 of the tile: 16-byte chunks 2 ct + g of a
         // 128-byte swizzled row (chunk c sits at c ^ (r % 8)); zero past the sequence or dv
         const bool tok = x.t0 + (long long)s * C64 + r < x.t1;
-        uint4 vc[3];
+        uint4 vc[2];
 #pragma unroll
-        for (int g = 0; g < 3; ++g) {
+        for (int g = 0; g < 2; ++g) {
             const int hf = r >> 5, rr = r & 31;
-            const int c = 3 * ch + g;
+            const int c = 2 * ct + g;
             vc[g] = (tok && 8 * g < nv)
                         ? *reinterpret_cast<const uint4*>(sm.vt[rs] + hf * 4096 + rr * 128 +
                                                          ((c ^ (rr & 7)) << 4))
@@ -808,16 +846,16 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
         }
         // B = beta V - w K S
         live = live && w64(ab, &sm.acc1_full[s & 1], (uint32_t)(s >> 1) & 1u);
-        float v[24];
+        float v[16];
 #pragma unroll
-        for (int j = 0; j < 24; ++j) v[j] = 0.f;
+        for (int j = 0; j < 16; ++j) v[j] = 0.f;
         if (live) {
             tc_fence_after();
-            ld_acc24s(tl + T_ACC1 + 96 * (s & 1) + j0, 0.f, v);
+            ld_acc16s(tl + T_ACC1 + 96 * (s & 1) + j0, 0.f, v);
         }
         warp_arrive64(&sm.acc1_free[s & 1], lane);
 #pragma unroll
-        for (int g = 0; g < 3; ++g) {
+        for (int g = 0; g < 2; ++g) {
             const uint32_t wd[4] = {vc[g].x, vc[g].y, vc[g].z, vc[g].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -826,18 +864,16 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
                 v[8 * g + 2 * e + 1] = bet * fv.y - wv * v[8 * g + 2 * e + 1];
             }
         }
-        put24s(sm.b_op, OPB, r, 3 * ch, C64, v, 1.f);
+        put16s(sm.b_op, OPB, r, 2 * ct, C64, v, 1.f);
         fence_async_smem();
         gbar(BAR_BD, BAR_BD_THREADS);  // B_s written: Delta(s)
         // Delta = -acc2 rows 0-63; D Delta
         live = live && w64(ab, &sm.acc2_full, (uint32_t)s & 1u);
         if (live) {
             tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < 24; ++j) v[j] = 0.f;
-            ld_acc24s(tl + T_ACC2 + j0, 0.f, v);
-            put24s(sm.d_op, OPB, r, 3 * ch, C64, v, -1.f);
-            put24s(sm.dd_op, OPB, r, 3 * ch, C64, v, -d);
+            ld_acc16s(tl + T_ACC2 + j0, 0.f, v);
+            put16s(sm.d_op, OPB, r, 2 * ct, C64, v, -1.f);
+            put16s(sm.dd_op, OPB, r, 2 * ct, C64, v, -d);
             fence_async_smem();
         }
         tc_fence_before();
@@ -925,7 +961,7 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], 2);      // G1 and the last P Delta product of the block
             mbar_init(&sm.acc1_full[i], 1);
-            mbar_init(&sm.acc1_free[i], 8);  // BD and output warps
+            mbar_init(&sm.acc1_free[i], 10);  // BD and output warps
         }
         mbar_init(&sm.acc2_full, 1);
         mbar_init(&sm.acc3_full, 1);
@@ -948,14 +984,12 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     if (warp < 8)
         s64_role(sm, x, warp, lane, init_state, final_state);
-    else if (warp < 16)
+    else if (warp < 18)
         ((warp & 3) < 2) ? bd_role(sm, x, warp, lane) : o64_role(sm, x, warp, lane, out);
-    else if (warp == 16)
-        load64_role(sm, x, lane, &tm_q, &tm_k, &tm_v);
     else if (warp == 18)
         d_issue_role(sm, x, lane);
-    else if (warp == 19)
-        g1_issue_role(sm, x, lane);
+    else
+        g1_issue_role(sm, x, lane, &tm_q, &tm_k, &tm_v);
 
     tc_fence_before();
     __syncthreads();
