@@ -736,19 +736,21 @@ __device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
         }
         __syncwarp();
         if (leader && live) live = s < 1 || w64(ab, &sm.acc3_free, (uint32_t)(s - 1) & 1u);
-        gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s and D Delta_s written
+        gbar(BAR_BD, BAR_BD_THREADS);  // D Delta_s written
         if (leader && live) {
-            {
-                tc_fence_after();
+            tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(x.tmem + T_ACC3, dadd64(d_kt, r * 32768 + ks * 2048),
-                             dadd64(d_dd, ks * 256), id_g3, ks > 0);
-                mma_commit(&sm.acc3_full);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(x.tmem + T_ACC3, dadd64(d_kt, r * 32768 + ks * 2048),
+                         dadd64(d_dd, ks * 256), id_g3, ks > 0);
+            mma_commit(&sm.acc3_full);
+        }
+        __syncwarp();
+        if (leader && live) live = s < 1 || w64(ab, &sm.acc4_free, (uint32_t)(s - 1) & 1u);
+        gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s written
+        if (leader && live) {
             // P Delta(s) right behind G3(s): it runs while the S group forms S_{s+1}
-            live = live && (s < 1 || w64(ab, &sm.acc4_free, (uint32_t)(s - 1) & 1u));
-            if (live) {
+            {
                 tc_fence_after();
                 tp_product(r, T_ACC4, d_d);
                 mma_commit(&sm.acc4_full);
@@ -867,17 +869,21 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
         put16s(sm.b_op, OPB, r, 2 * ct, C64, v, 1.f);
         fence_async_smem();
         gbar(BAR_BD, BAR_BD_THREADS);  // B_s written: Delta(s)
-        // Delta = -acc2 rows 0-63; D Delta
+        // Delta = -acc2 rows 0-63: D Delta first (G3, on the chain), then Delta (P Delta)
         live = live && w64(ab, &sm.acc2_full, (uint32_t)s & 1u);
         if (live) {
             tc_fence_after();
             ld_acc16s(tl + T_ACC2 + j0, 0.f, v);
-            put16s(sm.d_op, OPB, r, 2 * ct, C64, v, -1.f);
             put16s(sm.dd_op, OPB, r, 2 * ct, C64, v, -d);
             fence_async_smem();
         }
         tc_fence_before();
-        gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s written: G3(s), P Delta(s)
+        gbar(BAR_BD, BAR_BD_THREADS);  // D Delta_s written: G3(s)
+        if (live) {
+            put16s(sm.d_op, OPB, r, 2 * ct, C64, v, -1.f);
+            fence_async_smem();
+        }
+        gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s written: P Delta(s)
     }
 }
 
