@@ -163,25 +163,29 @@ struct alignas(1024) Prep64Smem {
         // swizzle (two TMA boxes of 32 rows each).  Dead once the Gram product and the
         // norms are done; the solve's arrays then take the space.
         uint8_t kq[2][16384];
+        // The coupling products Z live in A's dead blocks: the 16-level ones of 32-token
+        // half b in A's diagonal block at (32 b, 32 b) (read only by the forward
+        // substitution before them), the 32-level one in A's top-left quarter (dead once
+        // the 16-level couplings are done); the top-right quarter holds A_ba transposed.
         struct {
             float Am[C64][68];
             float Tm[C64][68];  // T = (I + A)^-1, stored with its zero upper triangle
-            float Zm[32][36];   // coupling products
         } w;
     };
     alignas(16) float beta[C64];
     alignas(16) float G[C64];   // G of tokens 32-63 still lacks the first half's total
     alignas(16) float G2[C64];  // the block's G times log2(e)
+    alignas(16) float G2r[C64]; // G2 - log2(r_k): a column's decay and key scale in one exponent
     alignas(16) float rk[C64];
     alignas(16) float rq[C64];
     uint64_t bar_tma, bar_mma;
     uint32_t tmem;
 };
-static_assert(sizeof(Prep64Smem) <= 44 * 1024, "five intra-block CTAs per SM");
+static_assert(sizeof(Prep64Smem) <= 37 * 1024, "six intra-block CTAs per SM");
 
 constexpr int PREP64_THREADS = 128;
 
-__global__ void __launch_bounds__(PREP64_THREADS, 5)
+__global__ void __launch_bounds__(PREP64_THREADS, 6)
 intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                const float* __restrict__ A_log, const float* __restrict__ dt_bias,
@@ -268,8 +272,14 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             float ss = sumsq_line(sm.kq[hf] + row * 128, row + 4 * hf);
             ss += __shfl_xor_sync(0xffffffffu, ss, 1);
             if (hf == 0) {
-                if (e == 0) sm.rk[row] = rsqrtf(ss + kNormEps);
-                else sm.rq[row - 64] = rsqrtf(ss + kNormEps) * rsqrtf((float)DK);
+                if (e == 0) {
+                    sm.rk[row] = rsqrtf(ss + kNormEps);
+                    // log2(r_k) = -log2(ss + eps) / 2
+                    sm.G2r[row] = (sm.G[row] + (row >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f +
+                                  0.5f * __log2f(ss + kNormEps);
+                } else {
+                    sm.rq[row - 64] = rsqrtf(ss + kNormEps) * rsqrtf((float)DK);
+                }
             }
         }
     }
@@ -300,17 +310,15 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int kc = 0; kc < kc_end; ++kc) {
             float v[8], p[8];
             tmem_ld8(tmem + lane_base64(warp) + 8 * kc, v);
-            const float4 g0 = *reinterpret_cast<const float4*>(&sm.G2[8 * kc]);
-            const float4 g1 = *reinterpret_cast<const float4*>(&sm.G2[8 * kc + 4]);
-            const float4 r0 = *reinterpret_cast<const float4*>(&sm.rk[8 * kc]);
-            const float4 r1 = *reinterpret_cast<const float4*>(&sm.rk[8 * kc + 4]);
+            const float4 g0 = *reinterpret_cast<const float4*>(&sm.G2r[8 * kc]);
+            const float4 g1 = *reinterpret_cast<const float4*>(&sm.G2r[8 * kc + 4]);
             const float gj[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            const float rj[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int jj = 8 * kc + e;
-                const float pv = f * ex2_approx(Gi2 - gj[e]) * rj[e] * v[e];
+                // e^{G_i - G_j} r_k,j = 2^{G2_i - G2r_j}
+                const float pv = f * ex2_approx(Gi2 - gj[e]) * v[e];
                 p[e] = (jj < i || (!arow && jj == i)) ? pv : 0.f;
             }
             if (arow) {
@@ -380,7 +388,7 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float4 t4 = *reinterpret_cast<const float4*>(&sm.w.Tm[o + m][o + jc]);
             z[0] += a_ * t4.x; z[1] += a_ * t4.y; z[2] += a_ * t4.z; z[3] += a_ * t4.w;
         }
-        *reinterpret_cast<float4*>(&sm.w.Zm[16 * bi + i][jc]) = make_float4(z[0], z[1], z[2], z[3]);
+        *reinterpret_cast<float4*>(&sm.w.Am[o + i][o + jc]) = make_float4(z[0], z[1], z[2], z[3]);
     }
     __syncthreads();
     {
@@ -393,7 +401,7 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll 8
         for (int m = 0; m < mend; ++m) {
             const float tv = sm.w.Tm[o + 16 + i][o + 16 + m];
-            const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Zm[16 * bi + m][jc]);
+            const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Am[o + m][o + jc]);
             t[0] += tv * z4.x; t[1] += tv * z4.y; t[2] += tv * z4.z; t[3] += tv * z4.w;
         }
         *reinterpret_cast<float4*>(&sm.w.Tm[o + 16 + i][o + jc]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
@@ -416,8 +424,8 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             z[0] += a_ * t0v.x; z[1] += a_ * t0v.y; z[2] += a_ * t0v.z; z[3] += a_ * t0v.w;
             z[4] += a_ * t1v.x; z[5] += a_ * t1v.y; z[6] += a_ * t1v.z; z[7] += a_ * t1v.w;
         }
-        *reinterpret_cast<float4*>(&sm.w.Zm[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
-        *reinterpret_cast<float4*>(&sm.w.Zm[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
+        *reinterpret_cast<float4*>(&sm.w.Am[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
+        *reinterpret_cast<float4*>(&sm.w.Am[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
     }
     __syncthreads();
     {
@@ -430,8 +438,8 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll 4
         for (int m = 0; m < 8 * warp + 8; ++m) {
             const float tv = sm.w.Tm[32 + i][32 + m];
-            const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Zm[m][j0]);
-            const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Zm[m][j0 + 4]);
+            const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0]);
+            const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0 + 4]);
             t[0] += tv * z0.x; t[1] += tv * z0.y; t[2] += tv * z0.z; t[3] += tv * z0.w;
             t[4] += tv * z1.x; t[5] += tv * z1.y; t[6] += tv * z1.z; t[7] += tv * z1.w;
         }
