@@ -194,6 +194,8 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Prep64Smem& sm = *reinterpret_cast<Prep64Smem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    // the state kernel may be scheduled as SMs drain; it waits for this grid's completion
+    grid_dep_launch_dependents();
     const int h = blockIdx.x % Hv;
     const long long f = blockIdx.x / Hv;
     int s, c;
@@ -957,6 +959,7 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     x.ws = ws;
     const int ncols = min(NT, DV - x.col0);
     if (x.n == 0) {  // empty sequence: the final state is the initial one
+        grid_dep_wait();
         if (final_state && tid < DK) {
             const size_t row = (((size_t)x.s * Hv + x.h) * DK + tid) * DV + x.col0;
             for (int j = 0; j < ncols; j += 4)
@@ -995,6 +998,9 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     x.tmem = sm.tmem_base;
+    // launched behind the intra-block kernel with programmatic serialization: its records
+    // (and everything before it in the stream) are visible only after this
+    grid_dep_wait();
 
     if (warp < 8)
         s64_role(sm, x, warp, lane, init_state, final_state);
@@ -1053,10 +1059,21 @@ cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t st
         p.cu_seqlens, p.T, p.nseq, p.Hk, p.Hv, p.erase, (uint8_t*)ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    state64_kernel<<<(unsigned)(p.nseq * p.Hv * NTILES), SP_THREADS, sizeof(Sp64Smem), stream>>>(
-        mq, mk, mv, (const uint8_t*)ws, p.init_state, p.out, p.final_state,
-        p.cu_seqlens, p.T, p.Hk, p.Hv);
-    return cudaGetLastError();
+    // programmatic serialization: the state kernel's CTAs are scheduled as the intra-block
+    // CTAs drain and set up while the last of them finish (each waits in grid_dep_wait)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.nseq * p.Hv * NTILES));
+    cfg.blockDim = dim3(SP_THREADS);
+    cfg.dynamicSmemBytes = sizeof(Sp64Smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, state64_kernel, mq, mk, mv, (const uint8_t*)ws,
+                              (const float*)p.init_state, p.out, p.final_state,
+                              (const int32_t*)p.cu_seqlens, p.T, p.Hk, p.Hv);
 }
 
 }  // namespace gdr

@@ -72,6 +72,30 @@ def test_prefill_varlen_grouped(form):
     _check_prefill(inp, form)
 
 
+@pytest.mark.parametrize("erase", [True, False])
+def test_prefill_varlen_around_64_token_blocks(erase):
+    """The tensor-core prefill steps its state 64 tokens at a time over two 32-token
+    solves: packed sequences one short of, at, and one past one and two blocks (and of
+    a solve), with Hk=3 key heads shared by Hv=6, nonzero initial states."""
+    inp = synth.make_inputs(1, 0, 3, 6, 128, 128, "bf16", seed=15, s0_std=0.05,
+                            seqlens=[63, 64, 65, 127, 128, 129, 31, 33, 2])
+    d = to_device(inp)
+    out, fin = gdr.prefill(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                           d["init_state"], d["cu_seqlens"], erase=erase)
+    torch.cuda.synchronize()
+    assert gdr.gdr_device_status() == gdr.GDR_OK
+    ro, rS = oracle_forward(inp, erase=erase)
+    assert_parity(_np(out), ro, TAU["bf16"], f"varlen 64-token edges o (erase={erase})")
+    assert_parity(_np(fin), rS, TAU["bf16"], f"varlen 64-token edges S (erase={erase})")
+
+
+@pytest.mark.parametrize("T", [64, 65, 191, 256])
+def test_prefill_dense_block_multiples(T):
+    """Dense batches of two sequences at and just past 64-token block multiples."""
+    inp = synth.make_inputs(2, T, 2, 4, 128, 128, "bf16", seed=16 + T, s0_std=0.05)
+    _check_prefill(inp, "chunked")
+
+
 def test_zero_length_returns_initial_state():
     inp = synth.make_inputs(3, 0, 2, 2, 128, 128, "bf16", seed=10, s0_std=0.1)
     for form in ("chunked", "recurrent"):
