@@ -38,23 +38,25 @@ constexpr int kConvSeg = 64;    // tokens per thread when the state is not updat
 constexpr int kConvThreads = 256;
 constexpr int kConvBatch = 8;   // tokens whose loads a thread issues together
 
-// Thread -> (sequence b, time segment, group of 8 channels).  Channels are the fastest
-// index, so a warp moves 512 contiguous bytes per token in 16-byte accesses.
-__device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+// Thread -> (sequence b, time segment, group of 4 channels).  Channels are the fastest
+// index, so a warp moves 256 contiguous bytes per token in 8-byte accesses.  (Eight
+// channels per thread took 128 registers, two CTAs per SM; four take 80, three CTAs:
+// 148 -> 142 us on x [1, 8192, 18432].)
+__device__ __forceinline__ void unpack4(const uint2 u, float (&f)[4]) {
+    const uint32_t w[2] = {u.x, u.y};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < 2; ++e) {
         const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
         f[2 * e] = v.x;
         f[2 * e + 1] = v.y;
     }
 }
 
-__global__ void __launch_bounds__(kConvThreads)
+__global__ void __launch_bounds__(kConvThreads, 3)
 short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ w,
                        const float* __restrict__ bias, const float* state_in, float* state_out,
                        __nv_bfloat16* __restrict__ y, int B, int T, int C, int seg) {
-    constexpr int G = 8;  // channels per thread
+    constexpr int G = 4;  // channels per thread
     const int groups = C / G;
     const int nseg = (T + seg - 1) / seg;
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -78,7 +80,7 @@ short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restr
     for (int j = 0; j < kConvW - 1; ++j) {
         const int t = t0 - (kConvW - 1) + j;
         if (t >= 0) {
-            unpack8(*reinterpret_cast<const uint4*>(x + ((size_t)b * T + t) * C + c), h[j]);
+            unpack4(*reinterpret_cast<const uint2*>(x + ((size_t)b * T + t) * C + c), h[j]);
         } else {
             // state[b][c][j'] holds the input at time j' - 3 of this call
             const int jj = t + (kConvW - 1);
@@ -90,9 +92,9 @@ short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restr
     const __nv_bfloat16* xp = x + ((size_t)b * T + t0) * C + c;
     __nv_bfloat16* yp = y + ((size_t)b * T + t0) * C + c;
     // one token: SiLU(conv) of input v against the window h, then shift v into the window
-    auto step = [&](const uint4 raw, __nv_bfloat16* dst) {
+    auto step = [&](const uint2 raw, __nv_bfloat16* dst) {
         float v[G];
-        unpack8(raw, v);
+        unpack4(raw, v);
         uint32_t o[G / 2];
 #pragma unroll
         for (int e = 0; e < G; e += 2) {
@@ -103,7 +105,7 @@ short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restr
             const __nv_bfloat162 pr = __floats2bfloat162_rn(silu_fast(a0), silu_fast(a1));
             o[e / 2] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        __stcs(reinterpret_cast<uint4*>(dst), make_uint4(o[0], o[1], o[2], o[3]));
+        __stcs(reinterpret_cast<uint2*>(dst), make_uint2(o[0], o[1]));
 #pragma unroll
         for (int e = 0; e < G; ++e) {
             h[0][e] = h[1][e];
@@ -116,15 +118,15 @@ short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restr
     int t = t0;
     for (; t + kConvBatch <= t1; t += kConvBatch, xp += (size_t)kConvBatch * C,
                                  yp += (size_t)kConvBatch * C) {
-        uint4 raw[kConvBatch];
+        uint2 raw[kConvBatch];
 #pragma unroll
         for (int u = 0; u < kConvBatch; ++u)
-            raw[u] = __ldcs(reinterpret_cast<const uint4*>(xp + (size_t)u * C));
+            raw[u] = __ldcs(reinterpret_cast<const uint2*>(xp + (size_t)u * C));
 #pragma unroll
         for (int u = 0; u < kConvBatch; ++u) step(raw[u], yp + (size_t)u * C);
     }
 #pragma unroll 1
-    for (; t < t1; ++t, xp += C, yp += C) step(__ldcs(reinterpret_cast<const uint4*>(xp)), yp);
+    for (; t < t1; ++t, xp += C, yp += C) step(__ldcs(reinterpret_cast<const uint2*>(xp)), yp);
     // The new state (the last three inputs) is written by the thread of segment 0, the one
     // that read the old state, so the state may be updated in place whatever the number of
     // segments: with T >= 3 it is read back from x, with T < 3 (one segment) it is the
@@ -133,7 +135,7 @@ short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restr
 #pragma unroll
         for (int j = 0; j < kConvW - 1; ++j) {
             if (T >= kConvW - 1)
-                unpack8(*reinterpret_cast<const uint4*>(
+                unpack4(*reinterpret_cast<const uint2*>(
                             x + ((size_t)b * T + T - (kConvW - 1) + j) * C + c),
                         h[j]);
 #pragma unroll
@@ -254,7 +256,7 @@ cudaError_t launch_short_conv_silu(const void* x, const float* w, const float* b
         return cudaSuccess;
     }
     const int seg = kConvSeg;
-    const long long total = (long long)B * ((T + seg - 1) / seg) * (C / 8);
+    const long long total = (long long)B * ((T + seg - 1) / seg) * (C / 4);
     const unsigned grid = (unsigned)((total + kConvThreads - 1) / kConvThreads);
     short_conv_silu_kernel<<<grid, kConvThreads, 0, stream>>>(
         (const __nv_bfloat16*)x, w, bias, state_in, state_out, (__nv_bfloat16*)y, B, T, C, seg);
