@@ -500,7 +500,9 @@ constexpr int O_PITCH = 52;             // floats: 208 B rows, 16-byte aligned
 //   10, 11, 14, 15 output group (accumulator rows 64-127): O = E Q S + P Delta, staged in
 //                  shared memory and written by one bulk copy per row segment (per-lane
 //                  stores to rows 24 KB apart would hold up the memory pipe that the
-//                  operand stores of the chain use)
+//                  operand stores of the chain use); block s's epilogue waits for G1(s+1)
+//                  to be issued, so that it overlaps the BD group's epilogue on the other
+//                  sub-partitions rather than the S group's and the G1 issue
 // The S and BD groups read nothing from global memory inside the loop: a named barrier
 // orders memory like membar.cta and so waits for a warp's global loads still in flight.
 //   18             issues Delta, K^T D Delta and P Delta (meets the BD group on BAR_BD);
@@ -522,7 +524,7 @@ struct alignas(1024) Sp64Smem {
     uint8_t dd_op[2 * OPB];         // diag(D) Delta
     float o_st[C64][O_PITCH];       // output rows of block s (pitch: conflict-free v4 stores)
     uint64_t full[2], empty[2];
-    uint64_t acc1_full[2], acc1_free[2], acc2_full;
+    uint64_t acc1_full[2], acc1_free[2], acc2_full, g1_issued;
     uint64_t acc3_full, acc3_free, acc4_full, acc4_free, drain_s, drain_d;
     uint32_t tmem_base;
     int abort;
@@ -688,6 +690,7 @@ __device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane, const CU
                              dadd64(d_s, ks * 256), id96, ks > 0);
                 mma_commit(&sm.acc1_full[x1]);
                 mma_commit(&sm.empty[r]);
+                if (s >= 1) mbar_arrive(&sm.g1_issued);
             }
             // block s + 1 into slot (s + 1) & 1, once block s - 1 is done with it
             if (live && s >= 1 && s + 1 < x.n) {
@@ -917,6 +920,9 @@ __device__ void o64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
         tc_fence_after();
         ld_acc24s(tl + T_ACC1 + 96 * (s & 1) + j0, 0.f, o);
         warp_arrive64(&sm.acc1_free[s & 1], lane);
+        // after G1(s + 1) was issued: the epilogue then overlaps the BD group's (other
+        // sub-partitions) rather than the S group's and the G1 issue
+        if (s + 1 < x.n && !w64(ab, &sm.g1_issued, (uint32_t)s & 1u)) break;
         if (!w64(ab, &sm.acc4_full, (uint32_t)s & 1u)) break;
         tc_fence_after();
         ld_acc24s(tl + T_ACC4 + j0, e, o);
@@ -981,6 +987,7 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&sm.acc1_free[i], 10);  // BD and output warps
         }
         mbar_init(&sm.acc2_full, 1);
+        mbar_init(&sm.g1_issued, 1);
         mbar_init(&sm.acc3_full, 1);
         mbar_init(&sm.acc3_free, 8);  // S warps
         mbar_init(&sm.acc4_full, 1);
