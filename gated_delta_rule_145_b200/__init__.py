@@ -82,6 +82,8 @@ def library():
             fn.restype = _I
         lib.gdr_device_status.argtypes = [_P]
         lib.gdr_device_status.restype = _I
+        lib.gdr_selftest_bounded_wait.argtypes = [_P]
+        lib.gdr_selftest_bounded_wait.restype = _I
         lib.gdr_status_string.argtypes = [_I]
         lib.gdr_status_string.restype = ctypes.c_char_p
         lib.gdr_release_workspace.argtypes = []
@@ -97,6 +99,12 @@ def gdr_status_string(status: int) -> str:
 def gdr_device_status(stream=None) -> int:
     """Synchronise `stream` and return the device-side status (GDR_OK or an error code)."""
     return library().gdr_device_status(_stream(stream))
+
+
+def gdr_selftest_bounded_wait(stream=None) -> int:
+    """Enqueue the failure-detection self-test (see include/gdr.h); gdr_device_status then
+    reports GDR_ERR_TIMEOUT once its bounded wait has given up."""
+    return library().gdr_selftest_bounded_wait(_stream(stream))
 
 
 def gdr_release_workspace() -> None:

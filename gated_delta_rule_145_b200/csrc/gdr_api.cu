@@ -389,6 +389,11 @@ int gdr_device_status(gdr_stream_t stream) {
     return v ? GDR_ERR_TIMEOUT : GDR_OK;
 }
 
+int gdr_selftest_bounded_wait(gdr_stream_t stream) {
+    return gdr::launch_bounded_wait_selftest((cudaStream_t)stream) == cudaSuccess ? GDR_OK
+                                                                                 : GDR_ERR_CUDA;
+}
+
 void gdr_release_workspace(void) { gdr::workspace_release(); }
 
 const char* gdr_status_string(int status) {

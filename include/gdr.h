@@ -336,6 +336,17 @@ GDR_API int gdr_gated_rmsnorm_f32(const float* o, const float* z, const float* w
 GDR_API int gdr_device_status(gdr_stream_t stream);
 
 /*
+ * Failure-detection self-test: enqueues one single-warp kernel whose thread waits on a
+ * shared-memory barrier that nothing completes, through the same bounded wait the
+ * tensor-core kernels use.  After the wait's limit (2 s) it gives up, records a timeout and
+ * lets the kernel exit; gdr_device_status on `stream` then returns GDR_ERR_TIMEOUT (and
+ * clears the record), and the context stays usable.  Returns GDR_OK once the kernel is
+ * enqueued, GDR_ERR_CUDA on a launch error.  No counterpart on the pages: it checks this
+ * library's failure path without faulting or hanging the GPU.
+ */
+GDR_API int gdr_selftest_bounded_wait(gdr_stream_t stream);
+
+/*
  * Returns the workspace memory cached by earlier gdr_prefill_chunked calls to the system
  * (every device's pool is trimmed to zero).  Memory still in use by enqueued work is
  * released once that work completes.  No counterpart on the pages: it manages this
