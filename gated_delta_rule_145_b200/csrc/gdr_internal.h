@@ -53,6 +53,7 @@ size_t prefill_tc64_workspace_bytes(const FwdParams& p);
 cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t stream);
 int read_and_clear_tc64_status();
 cudaError_t launch_bounded_wait_selftest(cudaStream_t stream);
+int read_and_clear_selftest_status();
 
 // Returns the cached workspace memory of every device to the system; prefill_tc.cu.
 void workspace_release();

@@ -1162,8 +1162,9 @@ int read_and_clear_tc_status() {
         cudaMemcpyToSymbol(g_tc_status, &zero, sizeof(int));
     }
     const int v64 = read_and_clear_tc64_status();
-    if (v64 < 0) return -1;
-    return v != 0 ? v : v64;
+    const int vst = read_and_clear_selftest_status();
+    if (v64 < 0 || vst < 0) return -1;
+    return v != 0 ? v : (v64 != 0 ? v64 : vst);
 }
 
 }  // namespace gdr

@@ -1025,23 +1025,7 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (tid == 0 && sm.abort) atomicExch(&g_tc64_status, 1);
 }
 
-// Failure-detection self-test: one thread waits on a barrier that nothing completes; the
-// bounded wait gives up after its limit and the timeout is recorded like any kernel's.
-__global__ void bounded_wait_selftest_kernel() {
-    __shared__ uint64_t bar;
-    if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
-        mbar_init_fence();
-        if (!mbar_wait(&bar, 0)) atomicExch(&g_tc64_status, 1);
-    }
-}
-
 }  // namespace
-
-cudaError_t launch_bounded_wait_selftest(cudaStream_t stream) {
-    bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>();
-    return cudaGetLastError();
-}
 
 int read_and_clear_tc64_status() {
     int v = 0;
