@@ -99,17 +99,17 @@ int check_segment_maps(FwdParams p, const float* phi, const float* nmap) {
     return GDR_OK;
 }
 
-// N (the run from S = 0) into nmap, then Phi (from S = I with v = 0) into phi; no outputs.
+// N (the run from S = 0) into nmap and Phi (from S = I with v = 0) into phi, over one set
+// of records; no outputs.
 cudaError_t segment_maps(FwdParams p, float* phi, float* nmap, cudaStream_t stream) {
     p.init_state = nullptr;
     p.out = nullptr;
-    p.final_state = nmap;
-    cudaError_t e = gdr::launch_prefill_tc(p, stream);
+    void* ws = nullptr;
+    cudaError_t e = gdr::workspace_alloc(&ws, gdr::prefill_tc64_workspace_bytes(p), stream);
     if (e != cudaSuccess) return e;
-    p.v_zero = 1;
-    p.init_identity = 1;
-    p.final_state = phi;
-    return gdr::launch_prefill_tc(p, stream);
+    e = gdr::launch_prefill_tc64_maps_ws(p, ws, phi, nmap, stream);
+    const cudaError_t f = cudaFreeAsync(ws, stream);
+    return e != cudaSuccess ? e : f;
 }
 
 }  // namespace

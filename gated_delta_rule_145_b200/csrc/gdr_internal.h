@@ -51,6 +51,8 @@ cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stre
 // segment-map passes (v = 0, S = I, or no outputs).
 size_t prefill_tc64_workspace_bytes(const FwdParams& p);
 cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t stream);
+cudaError_t launch_prefill_tc64_maps_ws(const FwdParams& p, void* ws, float* phi, float* nmap,
+                                        cudaStream_t stream);
 int read_and_clear_tc64_status();
 cudaError_t launch_bounded_wait_selftest(cudaStream_t stream);
 int read_and_clear_selftest_status();

@@ -1095,7 +1095,7 @@ void workspace_release() {
 }
 
 // The 64-token step kernels take the rule and its erase=False form with outputs.
-static bool uses_tc64(const FwdParams& p) { return p.out && !p.v_zero && !p.init_identity; }
+static bool uses_tc64(const FwdParams&) { return true; }
 
 size_t prefill_tc_workspace_bytes(const FwdParams& p) {
     if (uses_tc64(p)) return prefill_tc64_workspace_bytes(p);

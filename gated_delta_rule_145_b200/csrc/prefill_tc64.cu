@@ -621,6 +621,9 @@ __device__ __forceinline__ void ld_acc24s(uint32_t taddr, float sc, float (&v)[2
 
 struct Sp64Ctx {
     int s, h, kh, Hv, col0, n;
+    int v_zero;         // v = 0: B = -diag(w) K S (the segment map Phi)
+    int init_identity;  // S_0 = I (the segment map Phi) instead of init_state or zeros
+    bool has_out;       // outputs wanted (else no P Delta product and no output epilogue)
     long long t0, t1, rbase;
     const uint8_t* ws;
     uint32_t tmem;
@@ -640,7 +643,7 @@ __device__ void issue_loads(Sp64Smem& sm, const Sp64Ctx& x, int s, const CUtenso
                             const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
     const int r = s & 1;
     uint64_t* bar = &sm.full[r];
-    mbar_arrive_expect_tx(bar, 10u * 4096u + 2u * r64::PART + r64::VEC_BYTES);
+    mbar_arrive_expect_tx(bar, (x.v_zero ? 8u : 10u) * 4096u + 2u * r64::PART + r64::VEC_BYTES);
     const int y = (int)(x.t0 + (long long)s * C64);
 #pragma unroll 1
     for (int hf = 0; hf < 2; ++hf) {
@@ -651,8 +654,10 @@ __device__ void issue_loads(Sp64Smem& sm, const Sp64Ctx& x, int s, const CUtenso
         tma_load_2d(base + 8192, tm_q, xx, y, bar);
         tma_load_2d(base + 12288, tm_q, xx, y + 32, bar);
     }
-    tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, y, bar);
-    tma_load_2d(sm.vt[r] + 4096, tm_v, x.h * DV + x.col0, y + 32, bar);
+    if (!x.v_zero) {
+        tma_load_2d(sm.vt[r], tm_v, x.h * DV + x.col0, y, bar);
+        tma_load_2d(sm.vt[r] + 4096, tm_v, x.h * DV + x.col0, y + 32, bar);
+    }
     const uint8_t* rc = x.record(s);
     bulk_load(sm.rec[r], rc + r64::OFF_A, r64::PART, bar);
     bulk_load(sm.rec[r] + r64::PART, rc + r64::OFF_A + r64::PART, r64::PART, bar);
@@ -759,16 +764,17 @@ __device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
             mma_commit(&sm.acc3_full);
         }
         __syncwarp();
-        if (leader && live) live = s < 1 || w64(ab, &sm.acc4_free, (uint32_t)(s - 1) & 1u);
+        if (leader && live && x.has_out)
+            live = s < 1 || w64(ab, &sm.acc4_free, (uint32_t)(s - 1) & 1u);
         gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s written
         if (leader && live) {
             // P Delta(s) right behind G3(s): it runs while the S group forms S_{s+1}
-            {
+            if (x.has_out) {
                 tc_fence_after();
                 tp_product(r, T_ACC4, d_d);
                 mma_commit(&sm.acc4_full);
-                mma_commit(&sm.empty[r]);
             }
+            mma_commit(&sm.empty[r]);
         }
         __syncwarp();
     }
@@ -795,6 +801,11 @@ __device__ void s64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
     for (int j = 0; j < 24; j += 4) {
         float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
         if (init_state && j < nvalid) t = *reinterpret_cast<const float4*>(init_state + srow + j);
+        if (x.init_identity) {  // row k of I: a one in column k
+            const int c0 = x.col0 + j0 + j;
+            t = make_float4(k == c0 ? 1.f : 0.f, k == c0 + 1 ? 1.f : 0.f, k == c0 + 2 ? 1.f : 0.f,
+                            k == c0 + 3 ? 1.f : 0.f);
+        }
         Sm[j] = t.x; Sm[j + 1] = t.y; Sm[j + 2] = t.z; Sm[j + 3] = t.w;
     }
     put24s(sm.s_op, LO, k, 3 * ch, DK, Sm, 1.f);
@@ -848,7 +859,7 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
         const float d = sm.vec[rs][r64::VEC_D + r];
         // V row r, columns j0 .. j0 + 15 of the tile: 16-byte chunks 2 ct + g of a
         // 128-byte swizzled row (chunk c sits at c ^ (r % 8)); zero past the sequence or dv
-        const bool tok = x.t0 + (long long)s * C64 + r < x.t1;
+        const bool tok = !x.v_zero && x.t0 + (long long)s * C64 + r < x.t1;
         uint4 vc[2];
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
@@ -892,7 +903,7 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
         }
         tc_fence_before();
         gbar(BAR_BD, BAR_BD_THREADS);  // D Delta_s written: G3(s)
-        if (live) {
+        if (live && x.has_out) {
             put16s(sm.d_op, OPB, r, 2 * ct, C64, v, -1.f);
             fence_async_smem();
         }
@@ -909,6 +920,13 @@ __device__ void o64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
     const uint32_t tl = x.tmem + lane_base64(warp);
     const int nvalid = DV - (x.col0 + j0);
     int* ab = &sm.abort;
+    if (!x.has_out) {  // only release each Q S accumulator for G1's reuse
+        for (int s = 0; s < x.n; ++s) {
+            if (!w64(ab, &sm.acc1_full[s & 1], (uint32_t)(s >> 1) & 1u)) break;
+            warp_arrive64(&sm.acc1_free[s & 1], lane);
+        }
+        return;
+    }
     float e_next = x.vec(0)[r64::VEC_E + i];
     for (int s = 0; s < x.n; ++s) {
         const float e = e_next;
@@ -943,14 +961,28 @@ __device__ void o64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
     bulk_wait_all();
 }
 
+// kMap: the segment-map instance (flags at run time, gridDim.y = 2 runs N and Phi
+// together); the prefill instance has them fixed (v, outputs, init_state or zeros).
+template <bool kMap>
 __global__ void __launch_bounds__(SP_THREADS, 1)
 state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v,
                const uint8_t* __restrict__ ws,
                const float* init_state, float* __restrict__ out, float* final_state,
-               const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv) {
+               const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv, int v_zero,
+               int init_identity, float* phi) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Sp64Smem& sm = *reinterpret_cast<Sp64Smem*>(smem_raw);
+    if (!kMap) {
+        v_zero = 0;
+        init_identity = 0;
+    } else if (blockIdx.y == 1) {  // the second segment map of the same records: Phi
+        v_zero = 1;
+        init_identity = 1;
+        init_state = nullptr;
+        out = nullptr;
+        final_state = phi;
+    }
     const int tile = blockIdx.x % NTILES;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     Sp64Ctx x;
@@ -963,15 +995,24 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     x.n = (int)((x.t1 - x.t0 + C64 - 1) / C64);
     x.rbase = r64::block_base(cu_seqlens, x.s, T);
     x.ws = ws;
+    x.v_zero = v_zero;
+    x.init_identity = init_identity;
+    x.has_out = !kMap || out != nullptr;
     const int ncols = min(NT, DV - x.col0);
     if (x.n == 0) {  // empty sequence: the final state is the initial one
         grid_dep_wait();
         if (final_state && tid < DK) {
             const size_t row = (((size_t)x.s * Hv + x.h) * DK + tid) * DV + x.col0;
-            for (int j = 0; j < ncols; j += 4)
-                *reinterpret_cast<float4*>(final_state + row + j) =
-                    init_state ? *reinterpret_cast<const float4*>(init_state + row + j)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < ncols; j += 4) {
+                float4 t = init_state ? *reinterpret_cast<const float4*>(init_state + row + j)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                if (init_identity) {
+                    const int c0 = x.col0 + j;
+                    t = make_float4(tid == c0 ? 1.f : 0.f, tid == c0 + 1 ? 1.f : 0.f,
+                                    tid == c0 + 2 ? 1.f : 0.f, tid == c0 + 3 ? 1.f : 0.f);
+                }
+                *reinterpret_cast<float4*>(final_state + row + j) = t;
+            }
         }
         return;
     }
@@ -1043,33 +1084,45 @@ size_t prefill_tc64_workspace_bytes(const FwdParams& p) {
 
 // The rule and its erase=False form with outputs (bf16, dk = dv = 128, chunk 32), on a
 // caller's workspace of at least prefill_tc64_workspace_bytes(p).
-cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t stream) {
-    if (p.in != InType::BF16 || p.dk != DK || p.dv != DV || p.chunk != 32 || p.v_zero ||
-        p.init_identity || !p.out)
-        return cudaErrorNotSupported;
+namespace {
+
+struct Maps64 {
+    CUtensorMap q, k, v;
+};
+
+cudaError_t prepare64(const FwdParams& p, Maps64& m) {
     const long long tokens = p.cu_seqlens ? (long long)p.T : (long long)p.nseq * p.T;
     if (tokens <= 0 || tokens >= (1LL << 31) - 128) return cudaErrorNotSupported;
-    CUtensorMap mq, mk, mv;
-    if (!make_bf16_map(&mq, p.q, (uint64_t)p.Hk * DK, tokens) ||
-        !make_bf16_map(&mk, p.k, (uint64_t)p.Hk * DK, tokens) ||
-        !make_bf16_map(&mv, p.v, (uint64_t)p.Hv * DV, tokens))
+    if (!make_bf16_map(&m.q, p.q, (uint64_t)p.Hk * DK, tokens) ||
+        !make_bf16_map(&m.k, p.k, (uint64_t)p.Hk * DK, tokens) ||
+        !make_bf16_map(&m.v, p.v, (uint64_t)p.Hv * DV, tokens))
         return cudaErrorInvalidValue;
-    const long long nrec = r64::max_records(p.cu_seqlens != nullptr, p.nseq, p.T);
     cudaError_t e = cudaFuncSetAttribute(intra64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(Prep64Smem));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(state64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(state64_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sizeof(Sp64Smem));
     if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(state64_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(Sp64Smem));
+}
+
+cudaError_t launch_intra64(const FwdParams& p, const Maps64& m, void* ws, cudaStream_t stream) {
+    const long long nrec = r64::max_records(p.cu_seqlens != nullptr, p.nseq, p.T);
     intra64_kernel<<<(unsigned)(nrec * p.Hv), PREP64_THREADS, sizeof(Prep64Smem), stream>>>(
-        mq, mk, (const __nv_bfloat16*)p.a, (const __nv_bfloat16*)p.b, p.A_log, p.dt_bias,
+        m.q, m.k, (const __nv_bfloat16*)p.a, (const __nv_bfloat16*)p.b, p.A_log, p.dt_bias,
         p.cu_seqlens, p.T, p.nseq, p.Hk, p.Hv, p.erase, (uint8_t*)ws);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // programmatic serialization: the state kernel's CTAs are scheduled as the intra-block
-    // CTAs drain and set up while the last of them finish (each waits in grid_dep_wait)
+    return cudaGetLastError();
+}
+
+// The state pass over the records in ws.  With `dependent`, launched with programmatic
+// stream serialization behind the intra-block kernel: its CTAs are scheduled as the
+// intra-block CTAs drain and set up while the last of them finish (each then waits in
+// grid_dep_wait).
+cudaError_t launch_state64(const FwdParams& p, const Maps64& m, const void* ws, bool dependent,
+                           cudaStream_t stream, float* phi = nullptr) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.nseq * p.Hv * NTILES));
+    cfg.gridDim = dim3((unsigned)(p.nseq * p.Hv * NTILES), phi ? 2u : 1u);
     cfg.blockDim = dim3(SP_THREADS);
     cfg.dynamicSmemBytes = sizeof(Sp64Smem);
     cfg.stream = stream;
@@ -1077,10 +1130,51 @@ cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t st
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, state64_kernel, mq, mk, mv, (const uint8_t*)ws,
+    cfg.numAttrs = dependent ? 1 : 0;
+    const bool map = phi || p.v_zero || p.init_identity || !p.out;
+    return cudaLaunchKernelEx(&cfg, map ? state64_kernel<true> : state64_kernel<false>, m.q, m.k,
+                              m.v, (const uint8_t*)ws,
                               (const float*)p.init_state, p.out, p.final_state,
-                              (const int32_t*)p.cu_seqlens, p.T, p.Hk, p.Hv);
+                              (const int32_t*)p.cu_seqlens, p.T, p.Hk, p.Hv, p.v_zero,
+                              p.init_identity, phi);
+}
+
+}  // namespace
+
+// The rule and its erase=False form (bf16, dk = dv = 128, chunk 32), on a caller's
+// workspace of at least prefill_tc64_workspace_bytes(p).  Without outputs (p.out null) it
+// only carries the state; with v_zero and init_identity (both or neither, and no outputs)
+// it computes the segment map Phi of the rule.
+cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t stream) {
+    if (p.in != InType::BF16 || p.dk != DK || p.dv != DV || p.chunk != 32 ||
+        p.v_zero != p.init_identity || (p.v_zero && p.out) || (!p.erase && !p.out))
+        return cudaErrorNotSupported;
+    Maps64 m;
+    cudaError_t e = prepare64(p, m);
+    if (e != cudaSuccess) return e;
+    e = launch_intra64(p, m, ws, stream);
+    if (e != cudaSuccess) return e;
+    return launch_state64(p, m, ws, true, stream);
+}
+
+// Both segment maps of the rule over one set of records, in one state launch (gridDim.y
+// = 2): N (from S = 0) into nmap, and Phi (v = 0 from S = I) into phi; no outputs.
+cudaError_t launch_prefill_tc64_maps_ws(const FwdParams& p, void* ws, float* phi, float* nmap,
+                                        cudaStream_t stream) {
+    if (p.in != InType::BF16 || p.dk != DK || p.dv != DV || p.chunk != 32 || !p.erase)
+        return cudaErrorNotSupported;
+    FwdParams pn = p;
+    pn.init_state = nullptr;
+    pn.out = nullptr;
+    pn.final_state = nmap;
+    pn.v_zero = 0;
+    pn.init_identity = 0;
+    Maps64 m;
+    cudaError_t e = prepare64(pn, m);
+    if (e != cudaSuccess) return e;
+    e = launch_intra64(pn, m, ws, stream);
+    if (e != cudaSuccess) return e;
+    return launch_state64(pn, m, ws, true, stream, phi);
 }
 
 }  // namespace gdr
