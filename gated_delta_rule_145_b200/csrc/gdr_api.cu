@@ -1,7 +1,7 @@
 // gdr_api.cu -- the C ABI of libgdr.so (declared in include/gdr.h): argument checks,
 // then kernel launches.  Nothing is enqueued unless every check passes; no call
 // synchronises the stream.  The tensor-core prefill takes its workspace from a private
-// stream-ordered pool (prefill_tc.cu).
+// stream-ordered pool (workspace.cu).
 #include <cuda_runtime.h>
 #include <stdint.h>
 

@@ -33,22 +33,20 @@ cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
 // Chunked prefill on CUDA cores (any supported head size, fp32 or bf16); chunked_simt.cu.
 cudaError_t launch_chunked_simt(const FwdParams& p, cudaStream_t stream);
 
-// Chunked prefill on the tcgen05 tensor cores (bf16, dk = dv = 128, chunk 32):
-// the intra-chunk kernel, then the state-passing kernel, with a workspace of one record
-// per (chunk, value head) taken from the library's stream-ordered pool; prefill_tc.cu.
+// Chunked prefill on the tcgen05 tensor cores (bf16, dk = dv = 128, chunk 32): the
+// intra-block kernel, then the state-passing kernel, with a workspace of one record per
+// (64-token block, value head) taken from the library's stream-ordered pool; workspace.cu.
 // Returns cudaErrorNotSupported for shapes it does not handle.
 cudaError_t launch_prefill_tc(const FwdParams& p, cudaStream_t stream);
 
 // Bytes of workspace the tensor-core prefill needs for `p`, and the launch on a caller's
-// workspace of at least that size (16-byte aligned); prefill_tc.cu.  It runs the 64-token
-// step kernels of prefill_tc64.cu where they apply (the rule or its erase=False form with
-// outputs), the 32-token step kernels otherwise (the segment-map passes).
+// workspace of at least that size (16-byte aligned); workspace.cu.
 size_t prefill_tc_workspace_bytes(const FwdParams& p);
 cudaError_t launch_prefill_tc_ws(const FwdParams& p, void* ws, cudaStream_t stream);
 
 // The chunked prefill with the state advanced 64 tokens (two 32-token solve blocks) per
-// serial step: its workspace and launch; prefill_tc64.cu.  cudaErrorNotSupported for the
-// segment-map passes (v = 0, S = I, or no outputs).
+// serial step: its workspace and launch (also without outputs, or as the segment map
+// Phi: v = 0 from S = I), and both segment maps over one set of records; prefill_tc64.cu.
 size_t prefill_tc64_workspace_bytes(const FwdParams& p);
 cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t stream);
 cudaError_t launch_prefill_tc64_maps_ws(const FwdParams& p, void* ws, float* phi, float* nmap,
@@ -57,7 +55,7 @@ int read_and_clear_tc64_status();
 cudaError_t launch_bounded_wait_selftest(cudaStream_t stream);
 int read_and_clear_selftest_status();
 
-// Returns the cached workspace memory of every device to the system; prefill_tc.cu.
+// Returns the cached workspace memory of every device to the system; workspace.cu.
 void workspace_release();
 
 // The steps around the rule (mixer_io.cu): the four-tap causal convolution + SiLU on bf16
@@ -82,7 +80,7 @@ cudaError_t launch_segment_bounds(int32_t* cu, int G, int L, int T, cudaStream_t
 cudaError_t launch_prefill_host(const FwdParams& host_params, int seg, cudaStream_t stream,
                                 int (*prefill)(const FwdParams&, cudaStream_t), int* status);
 
-// The library's stream-ordered workspace pool (prefill_tc.cu).
+// The library's stream-ordered workspace pool (workspace.cu).
 cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
 
 // The fixed scratch area of the no-allocation prefill entry point: its size, and its
@@ -90,8 +88,8 @@ cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** ptr);
 
-// Reads and clears the tensor-core kernels' timeout record (nonzero if set, 0 if not,
-// -1 on a CUDA error); prefill_tc.cu.
+// Reads and clears the tensor-core kernels' and the self-test's timeout records (nonzero if
+// set, 0 if not, -1 on a CUDA error); workspace.cu.
 int read_and_clear_tc_status();
 
 }  // namespace gdr

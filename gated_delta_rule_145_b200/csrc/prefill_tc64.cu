@@ -19,8 +19,10 @@
 // T = [[T_a, 0], [-T_b A_ba T_a, T_b]].  The chunk size of the solve is 32; the state
 // passes over two solve blocks per step.
 //
-// Precision.  As in prefill_tc.cu: products have a raw bf16 operand or split an fp32
-// operand into bf16 hi + lo; derived x derived products take hi*hi + hi*lo + lo*hi.
+// Precision.  Every tensor-core product has a raw bf16 operand (K, Q, V) or splits an fp32
+// operand into bf16 hi + lo (about 16 significant bits); a product of two derived operands
+// takes hi*hi + hi*lo + lo*hi (here lo*lo too, at no extra instruction).  Dropping any one lo
+// part moves the result by ~1e-2 of its RMS at the workload sizes, against a 2e-3 bound.
 //
 // Kernels:
 //   intra64_kernel  one CTA per (64-token block, value head): gates, norms, the Gram

@@ -2,13 +2,12 @@
 the oracle's sequential recurrence.
 
 The kernels keep raw K, Q, V as tensor-core operands and move normalisation and decay
-into per-chunk C x C matrices and row scales (the chunk record), then run the chain
-with one chunk of lookahead (the state enters Delta_{c+1} through Y_{c+1} = gamma_c
-K_{c+1} S_c, a chunk early).  This test writes that restatement out from its formulas --
+into per-block matrices and row scales (the block record), then step the state 64 tokens
+at a time over two 32-token solves.  This test writes that step out from its formulas --
 nothing here is shared with the CUDA code -- and requires it to reproduce the oracle to
-rounding, for the rule and for its erase=False form, with a ragged last chunk.  A slip
-in the restated algebra (a sign, a missing decay factor, a misplaced row scale) fails
-here without a GPU.
+rounding, for the rule and for its erase=False form, with a ragged last block.  A slip
+in the restated algebra (a sign, a missing decay factor, a misplaced row scale, the
+coupling of the two solves) fails here without a GPU.
 """
 
 import numpy as np
@@ -17,75 +16,6 @@ import pytest
 from gated_delta_rule_145_b200 import synth
 
 EPS = 1e-6
-
-
-def _records(Kc, Qc, beta, g, erase):
-    """The per-chunk quantities of the chunk record, from raw rows of one chunk."""
-    C, dk = Kc.shape
-    rk = 1.0 / np.sqrt((Kc * Kc).sum(1) + EPS)
-    rq = 1.0 / np.sqrt((Qc * Qc).sum(1) + EPS) / np.sqrt(dk)
-    G = np.cumsum(g)
-    lower = np.tril(np.ones((C, C), dtype=bool))
-    dec = np.where(lower, np.exp(np.where(lower, G[:, None] - G[None, :], 0.0)), 0.0)
-    KK = Kc @ Kc.T
-    A = np.where(np.tril(lower, -1), beta[:, None] * dec * rk[:, None] * rk[None, :] * KK, 0.0)
-    if not erase:
-        A = np.zeros_like(A)
-    T = np.linalg.inv(np.eye(C) + A)
-    w = beta * np.exp(G) * rk if erase else np.zeros(C)
-    return dict(
-        Wt=T * w[None, :], Tb=T * beta[None, :],
-        P=dec * rq[:, None] * rk[None, :] * (Qc @ Kc.T),
-        E=np.exp(G) * rq, D=np.exp(G[-1] - G) * rk, gamma=np.exp(G[-1]))
-
-
-def _lookahead_prefill(q, k, v, beta, g, S0, C, erase):
-    """One (sequence, head): q, k [T, dk], v [T, dv] raw; returns (o, S_T)."""
-    T, dk = k.shape
-    n = -(-T // C)
-    pad = n * C - T
-    # padding rows: no decay, no write, zero K / Q / V (as the kernels treat them)
-    padz = lambda x: np.concatenate([x, np.zeros((pad,) + x.shape[1:])]) if pad else x
-    q, k, v, beta, g = (padz(x) for x in (q, k, v, beta, g))
-    chunks = [slice(c * C, (c + 1) * C) for c in range(n)]
-    R = [_records(k[s], q[s], beta[s], g[s], erase) for s in chunks]
-    K = [k[s] for s in chunks]
-    Q = [q[s] for s in chunks]
-    V = [v[s] for s in chunks]
-    o = np.zeros((n * C, v.shape[1]))
-    S = S0.copy()
-    delta = R[0]["Tb"] @ V[0] - R[0]["Wt"] @ (K[0] @ S)
-    for c in range(n):
-        o[chunks[c]] = R[c]["E"][:, None] * (Q[c] @ S) + R[c]["P"] @ delta
-        if c + 1 < n:
-            # lookahead: Y_{c+1} from S_c, M_{c+1} couples Delta_{c+1} to Delta_c
-            Y = R[c]["gamma"] * (K[c + 1] @ S)
-            M = R[c + 1]["Wt"] @ (K[c + 1] @ K[c].T) * R[c]["D"][None, :]
-            nxt = R[c + 1]["Tb"] @ V[c + 1] - R[c + 1]["Wt"] @ Y - M @ delta
-        S = R[c]["gamma"] * S + K[c].T @ (R[c]["D"][:, None] * delta)
-        if c + 1 < n:
-            delta = nxt
-    return o[:T], S
-
-
-@pytest.mark.parametrize("erase", [True, False])
-@pytest.mark.parametrize("T,C", [(23, 4), (32, 8), (5, 8)])
-def test_lookahead_chunk_algebra_matches_the_recurrence(erase, T, C):
-    from oracle import oracle
-
-    inp = synth.make_inputs(1, T, 2, 4, 8, 8, "f32", seed=300 + T + C, s0_std=0.3)
-    ro, rS = oracle.forward(inp.q, inp.k, inp.v, inp.a, inp.b, inp.A_log, inp.dt_bias,
-                            inp.init_state, erase=erase)
-    _, _, g, beta = oracle.prepare(inp.q, inp.k, inp.a, inp.b, inp.A_log, inp.dt_bias)
-    grp = 4 // 2
-    for h in range(4):
-        kh = h // grp
-        o, S = _lookahead_prefill(inp.q[0, :, kh].astype(np.float64),
-                                  inp.k[0, :, kh].astype(np.float64),
-                                  inp.v[0, :, h].astype(np.float64), beta[0, :, h], g[0, :, h],
-                                  inp.init_state[0, h].astype(np.float64), C, erase)
-        np.testing.assert_allclose(o, ro[0, :, h], rtol=1e-9, atol=1e-11)
-        np.testing.assert_allclose(S, rS[0, h], rtol=1e-9, atol=1e-11)
 
 
 @pytest.mark.parametrize("erase", [True, False])
