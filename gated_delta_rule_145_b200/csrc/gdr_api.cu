@@ -197,8 +197,20 @@ int gdr_prefill_chunked_cp(const void* q, const void* k, const void* v, const vo
     FwdParams sp = p;
     sp.cu_seqlens = cu;
     sp.nseq = G;
+    void* rec = nullptr;
+    e = gdr::workspace_alloc(&rec, gdr::prefill_tc64_workspace_bytes(sp), st);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(ws, st);
+        return to_status(e);
+    }
+    // one set of intra-block records serves the maps and the prefill of the segments
     e = gdr::launch_segment_bounds(cu, G, L, T, st);
-    if (e == cudaSuccess) e = segment_maps(sp, phi, nmap, st);
+    if (e == cudaSuccess) {
+        FwdParams mp = sp;
+        mp.init_state = nullptr;
+        mp.out = nullptr;
+        e = gdr::launch_prefill_tc64_maps_ws(mp, rec, phi, nmap, st);
+    }
     if (e == cudaSuccess)
         e = gdr::launch_segment_combine(phi, nmap, init_state, seg_init, final_state, G, Hv, 128,
                                         st);
@@ -206,10 +218,11 @@ int gdr_prefill_chunked_cp(const void* q, const void* k, const void* v, const vo
         sp.init_state = seg_init;
         sp.out = out;
         sp.final_state = nullptr;
-        e = gdr::launch_prefill_tc(sp, st);
+        e = gdr::launch_prefill_tc64_state_ws(sp, rec, st);
     }
-    const cudaError_t f = cudaFreeAsync(ws, st);
-    return to_status(e != cudaSuccess ? e : f);
+    const cudaError_t f = cudaFreeAsync(rec, st);
+    const cudaError_t f2 = cudaFreeAsync(ws, st);
+    return to_status(e != cudaSuccess ? e : f != cudaSuccess ? f : f2);
 }
 
 int gdr_prefill_chunked_host(const void* q, const void* k, const void* v, const void* a,

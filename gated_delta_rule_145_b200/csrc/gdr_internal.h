@@ -51,6 +51,11 @@ size_t prefill_tc64_workspace_bytes(const FwdParams& p);
 cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t stream);
 cudaError_t launch_prefill_tc64_maps_ws(const FwdParams& p, void* ws, float* phi, float* nmap,
                                         cudaStream_t stream);
+// The state pass with outputs over records already in ws (from either launch above on the
+// same q, k, gates and sequence bounds), launched as a programmatic dependent of the grid
+// before it in the stream.
+cudaError_t launch_prefill_tc64_state_ws(const FwdParams& p, const void* ws,
+                                         cudaStream_t stream);
 int read_and_clear_tc64_status();
 cudaError_t launch_bounded_wait_selftest(cudaStream_t stream);
 int read_and_clear_selftest_status();

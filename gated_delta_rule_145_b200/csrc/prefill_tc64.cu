@@ -1159,6 +1159,22 @@ cudaError_t launch_prefill_tc64_ws(const FwdParams& p, void* ws, cudaStream_t st
     return launch_state64(p, m, ws, true, stream);
 }
 
+// The state pass alone (the rule with outputs) over the records that an earlier launch
+// wrote into ws for the same q, k, gates and sequence bounds: the records depend on
+// neither v nor the start state.  Launched with programmatic stream serialization behind
+// the grid before it, which must let it start (griddepcontrol.launch_dependents) no earlier
+// than it is safe to set up: the state kernel reads nothing before its grid_dep_wait.
+cudaError_t launch_prefill_tc64_state_ws(const FwdParams& p, const void* ws,
+                                         cudaStream_t stream) {
+    if (p.in != InType::BF16 || p.dk != DK || p.dv != DV || p.chunk != 32 || !p.erase ||
+        p.v_zero || p.init_identity || !p.out)
+        return cudaErrorNotSupported;
+    Maps64 m;
+    const cudaError_t e = prepare64(p, m);
+    if (e != cudaSuccess) return e;
+    return launch_state64(p, m, ws, true, stream);
+}
+
 // Both segment maps of the rule over one set of records, in one state launch (gridDim.y
 // = 2): N (from S = 0) into nmap, and Phi (v = 0 from S = I) into phi; no outputs.
 cudaError_t launch_prefill_tc64_maps_ws(const FwdParams& p, void* ws, float* phi, float* nmap,

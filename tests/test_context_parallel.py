@@ -199,10 +199,11 @@ def test_segment_maps_match_oracle():
 
 
 @pytest.mark.gpu
-def test_segment_combine_matches_composition():
+@pytest.mark.parametrize("Hv", [3, 12, 30, 48])  # slices of 8, 16, 32, 64 columns on 148 SMs
+def test_segment_combine_matches_composition(Hv):
     torch = pytest.importorskip("torch")
-    rng = np.random.default_rng(7)
-    G, Hv, d = 5, 3, 128
+    rng = np.random.default_rng(7 + Hv)
+    G, d = 5, 128
     # contractive maps, as the rule's are (|Phi| <= 1): scaled random matrices
     phi = rng.standard_normal((G, Hv, d, d)) * (0.9 / np.sqrt(d))
     nmap = rng.standard_normal((G, Hv, d, d))
