@@ -71,6 +71,8 @@ cudaError_t launch_short_conv_silu(const void* x, const float* w, const float* b
                                    int C, cudaStream_t stream);
 cudaError_t launch_gated_rmsnorm(const float* o, const void* z, bool z_f32, const float* weight,
                                  float* y, long long rows, int d, float eps, cudaStream_t stream);
+// Reads and clears the tiled convolution's timeout record (nonzero if set, -1 on error).
+int read_and_clear_conv_status();
 
 // Composition of per-segment state maps, and segment boundaries of one sequence cut into
 // G segments of L tokens; segments.cu.
@@ -93,8 +95,8 @@ cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** ptr);
 
-// Reads and clears the tensor-core kernels' and the self-test's timeout records (nonzero if
-// set, 0 if not, -1 on a CUDA error); workspace.cu.
+// Reads and clears the tensor-core kernels', the tiled convolution's and the self-test's
+// timeout records (nonzero if set, 0 if not, -1 on a CUDA error); workspace.cu.
 int read_and_clear_tc_status();
 
 }  // namespace gdr

@@ -17,19 +17,36 @@
 //          without one; the state after the call holds the last three inputs.
 //   norm   y = o / sqrt(mean_d(o^2) + eps) * weight * SiLU(z), weight shared by heads.
 // Both are HBM-bound streaming passes: coalesced vector loads, streaming stores, no reuse.
+// The convolution of long inputs streams x through shared memory by TMA (a ring of tiles
+// per CTA, so the bytes in flight do not depend on registers); short inputs (decode steps)
+// take a per-thread kernel that reads only the rows it needs.
 #include <algorithm>
 
 #include "gdr_common.cuh"
 #include "gdr_internal.h"
+#include "tcgen05.cuh"
+#include "tma_map.h"
 
 namespace gdr {
+
+// Set when a bounded wait of the tiled convolution gave up (read and cleared by
+// read_and_clear_conv_status(), reported by gdr_device_status()).
+__device__ int g_conv_status = 0;
+
 namespace {
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
 
-// SiLU with the fast exponential and division (relative error ~1e-6): for bf16 outputs,
-// whose rounding step is 2^-8, this keeps the pass bound by memory, not by arithmetic.
-__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+// SiLU for bf16 outputs (rounding step 2^-8) from the special-function unit's 2^x and
+// reciprocal in their flush-to-zero forms, x * 1 / (1 + 2^(-x log2 e)), relative error
+// ~1e-6; five instructions, so the pass stays bound by memory.  Below x = -88, 2^(...)
+// is +inf, its reciprocal 0 and SiLU -0.
+__device__ __forceinline__ float silu_fast(float x) {
+    float e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * -1.4426950408889634f));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+    return x * r;
+}
 
 // ------------------------------------------------------------------------ conv + SiLU
 
@@ -145,6 +162,196 @@ short_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, const float* __restr
     }
 }
 
+// Tiled form for long inputs.  CTA -> (channel tile of 128, sequence b, time segment);
+// a producer warp streams the segment's tiles of 64 tokens x 128 channels (16 KB, one TMA
+// box) into a four-slot ring; consumer warp w convolves tile rows 8 w .. 8 w + 7, lane ->
+// four channels, with the three rows before its first one read from the same tile (warp
+// 0: from the previous tile, which is released only after the next one is consumed).
+constexpr int kCvCh = 128;
+constexpr int kCvRows = 64;
+constexpr int kCvStages = 4;
+constexpr int kCvWarps = 8;
+constexpr int kCvThreads = 32 * (kCvWarps + 1);
+constexpr uint32_t kCvTile = kCvRows * kCvCh * 2;
+constexpr int kCvMinT = 256;  // shorter inputs take the per-thread kernel
+
+struct alignas(128) ConvSmem {
+    uint8_t tile[kCvStages][kCvTile];
+    uint64_t full[kCvStages], empty[kCvStages];
+};
+
+// Four bf16 channels from 8 bytes of shared memory as two fp32 pairs.
+__device__ __forceinline__ void lds_unpack2x2(const uint8_t* p, float2 (&f)[2]) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    f[0] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    f[1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+}
+
+// silu_fast on a pair, the multiplies and the add as paired fp32 instructions
+__device__ __forceinline__ float2 silu_fast2(float2 a) {
+    const float2 m = __fmul2_rn(a, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+    float2 e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e.x) : "f"(m.x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e.y) : "f"(m.y));
+    const float2 d = __fadd2_rn(e, make_float2(1.f, 1.f));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.x) : "f"(d.x));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.y) : "f"(d.y));
+    return __fmul2_rn(a, r);
+}
+
+__global__ void __launch_bounds__(kCvThreads, 3)
+short_conv_silu_tiled_kernel(const __grid_constant__ CUtensorMap tm_x,
+                             const __nv_bfloat16* __restrict__ x, const float* __restrict__ w,
+                             const float* __restrict__ bias, const float* state_in,
+                             float* state_out, __nv_bfloat16* __restrict__ y, int T, int C,
+                             int nct, int nseg, int segT) {
+    using namespace tc;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    ConvSmem& sm = *reinterpret_cast<ConvSmem*>(smem_raw);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int ct = blockIdx.x % nct, rest = blockIdx.x / nct;
+    const int sg = rest % nseg, b = rest / nseg;
+    const int t0 = sg * segT, t1 = min(T, t0 + segT);
+    const int ntile = (t1 - t0 + kCvRows - 1) / kCvRows;
+    const int c0 = ct * kCvCh;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kCvStages; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], kCvWarps);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (warp == kCvWarps) {  // producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < ntile; ++i) {
+                const int st = i % kCvStages;
+                // the slot's previous tile (i - 4) is released once tile i - 3 is consumed
+                if (i >= kCvStages &&
+                    !mbar_wait(&sm.empty[st], (uint32_t)(i / kCvStages - 1) & 1u)) {
+                    atomicExch(&g_conv_status, 1);
+                    break;
+                }
+                mbar_arrive_expect_tx(&sm.full[st], kCvTile);
+                tma_load_2d(sm.tile[st], &tm_x, c0, b * T + t0 + kCvRows * i, &sm.full[st]);
+                issued = i + 1;
+            }
+            // every copy started here has landed before the CTA may exit
+            for (int i = max(0, issued - kCvStages); i < issued; ++i)
+                mbar_wait(&sm.full[i % kCvStages], (uint32_t)(i / kCvStages) & 1u);
+        }
+        return;
+    }
+    const int c = c0 + 4 * lane;
+    const bool cvalid = c < C;  // C is a multiple of 8: a group is wholly in or out
+    // channel pairs (c, c + 1) and (c + 2, c + 3): taps, bias, window
+    float2 wt[2][kConvW], bs[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        const float4 u = cvalid ? *reinterpret_cast<const float4*>(w + (size_t)(c + 2 * p) * kConvW)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v = cvalid
+                             ? *reinterpret_cast<const float4*>(w + (size_t)(c + 2 * p + 1) * kConvW)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        wt[p][0] = make_float2(u.x, v.x);
+        wt[p][1] = make_float2(u.y, v.y);
+        wt[p][2] = make_float2(u.z, v.z);
+        wt[p][3] = make_float2(u.w, v.w);
+        bs[p] = (bias && cvalid) ? make_float2(bias[c + 2 * p], bias[c + 2 * p + 1])
+                                 : make_float2(0.f, 0.f);
+    }
+    // warp 0's window before the segment: x rows t0 - 3 .. t0 - 1, or the state at t0 = 0
+    float2 h[kConvW - 1][2];
+#pragma unroll
+    for (int j = 0; j < kConvW - 1; ++j) h[j][0] = h[j][1] = make_float2(0.f, 0.f);
+    if (warp == 0 && cvalid) {
+#pragma unroll
+        for (int j = 0; j < kConvW - 1; ++j) {
+            const int t = t0 - (kConvW - 1) + j;
+            if (t >= 0) {
+                float f[4];
+                unpack4(*reinterpret_cast<const uint2*>(x + ((size_t)b * T + t) * C + c), f);
+                h[j][0] = make_float2(f[0], f[1]);
+                h[j][1] = make_float2(f[2], f[3]);
+            } else if (state_in) {
+                const float* sp = state_in + ((size_t)b * C + c) * (kConvW - 1) + t + kConvW - 1;
+                h[j][0] = make_float2(sp[0], sp[kConvW - 1]);
+                h[j][1] = make_float2(sp[2 * (kConvW - 1)], sp[3 * (kConvW - 1)]);
+            }
+        }
+    }
+    const int r0 = 8 * warp;
+    const uint32_t lo = 8u * (uint32_t)lane;  // this lane's bytes in a 256-byte tile row
+    for (int i = 0; i < ntile; ++i) {
+        const int st = i % kCvStages;
+        if (!mbar_wait(&sm.full[st], (uint32_t)(i / kCvStages) & 1u)) {
+            if (lane == 0) atomicExch(&g_conv_status, 1);
+            break;
+        }
+        const uint8_t* tl = sm.tile[st];
+        if (warp > 0) {
+#pragma unroll
+            for (int j = 0; j < kConvW - 1; ++j) lds_unpack2x2(tl + (r0 - 3 + j) * 256 + lo, h[j]);
+        } else if (i > 0) {
+            const uint8_t* pv = sm.tile[(i - 1) % kCvStages];
+#pragma unroll
+            for (int j = 0; j < kConvW - 1; ++j)
+                lds_unpack2x2(pv + (kCvRows - 3 + j) * 256 + lo, h[j]);
+        }
+        const int tb = t0 + kCvRows * i + r0;
+        __nv_bfloat16* yp = y + ((size_t)b * T + tb) * C + c;
+        // one row: SiLU(conv) against the window, stored, then shifted into the window
+        auto row = [&](int rr) {
+            float2 v[2];
+            lds_unpack2x2(tl + (r0 + rr) * 256 + lo, v);
+            uint32_t o[2];
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                // the same fused multiply-adds, in the same order, as the per-thread kernel
+                float2 a = __ffma2_rn(wt[p][0], h[0][p], bs[p]);
+                a = __ffma2_rn(wt[p][1], h[1][p], a);
+                a = __ffma2_rn(wt[p][2], h[2][p], a);
+                a = __ffma2_rn(wt[p][3], v[p], a);
+                const float2 sv = silu_fast2(a);
+                const __nv_bfloat162 pr = __floats2bfloat162_rn(sv.x, sv.y);
+                o[p] = *reinterpret_cast<const uint32_t*>(&pr);
+            }
+            if (cvalid) __stcs(reinterpret_cast<uint2*>(yp + (size_t)rr * C), make_uint2(o[0], o[1]));
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                h[0][p] = h[1][p];
+                h[1][p] = h[2][p];
+                h[2][p] = v[p];
+            }
+        };
+        if (tb + 8 <= t1) {  // all eight rows in the segment: no per-row test
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) row(rr);
+        } else {
+#pragma unroll 1
+            for (int rr = 0; rr < t1 - tb; ++rr) row(rr);
+        }
+        __syncwarp();
+        // tile i - 1 is no longer needed by anyone once tile i is done
+        if (i > 0 && lane == 0) mbar_arrive(&sm.empty[(i - 1) % kCvStages]);
+    }
+    // the new state (the last three inputs, T >= 3 here) by the threads that read the old
+    // one, so the state may be updated in place
+    if (state_out && sg == 0 && warp == 0 && cvalid) {
+#pragma unroll
+        for (int j = 0; j < kConvW - 1; ++j) {
+            float v[4];
+            unpack4(*reinterpret_cast<const uint2*>(
+                        x + ((size_t)b * T + T - (kConvW - 1) + j) * C + c),
+                    v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                state_out[((size_t)b * C + c + e) * (kConvW - 1) + j] = v[e];
+        }
+    }
+}
+
 // ---------------------------------------------------------------------- gated RMSNorm
 
 constexpr int kNormThreads = 256;
@@ -255,12 +462,45 @@ cudaError_t launch_short_conv_silu(const void* x, const float* w, const float* b
             return cudaMemsetAsync(state_out, 0, sizeof(float) * B * C * (kConvW - 1), stream);
         return cudaSuccess;
     }
+    if (T >= kCvMinT) {
+        // one wave of three CTAs per SM: channel tiles x sequences x time segments
+        const int nct = (C + kCvCh - 1) / kCvCh;
+        const long long want = 3LL * sm_count();
+        const long long per_seq = std::max<long long>(1, want / ((long long)B * nct));
+        const int tiles = (T + kCvRows - 1) / kCvRows;
+        const int nseg0 = (int)std::min<long long>(per_seq, tiles);
+        const int segT = (tiles + nseg0 - 1) / nseg0 * kCvRows;
+        const int nseg = (T + segT - 1) / segT;
+        const long long grid = (long long)nct * B * nseg;
+        CUtensorMap tm;
+        if (grid < 0x7fffffffLL && (long long)B * T < 0x7fffffffLL &&
+            make_bf16_map_plain(&tm, x, (uint64_t)C, (uint64_t)B * T, kCvCh, kCvRows)) {
+            cudaError_t e = cudaFuncSetAttribute(short_conv_silu_tiled_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)sizeof(ConvSmem));
+            if (e != cudaSuccess) return e;
+            short_conv_silu_tiled_kernel<<<(unsigned)grid, kCvThreads, sizeof(ConvSmem), stream>>>(
+                tm, (const __nv_bfloat16*)x, w, bias, state_in, state_out, (__nv_bfloat16*)y, T,
+                C, nct, nseg, segT);
+            return cudaGetLastError();
+        }
+    }
     const int seg = kConvSeg;
     const long long total = (long long)B * ((T + seg - 1) / seg) * (C / 4);
     const unsigned grid = (unsigned)((total + kConvThreads - 1) / kConvThreads);
     short_conv_silu_kernel<<<grid, kConvThreads, 0, stream>>>(
         (const __nv_bfloat16*)x, w, bias, state_in, state_out, (__nv_bfloat16*)y, B, T, C, seg);
     return cudaGetLastError();
+}
+
+int read_and_clear_conv_status() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_conv_status, sizeof(int)) != cudaSuccess) return -1;
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_conv_status, &zero, sizeof(int));
+    }
+    return v;
 }
 
 cudaError_t launch_gated_rmsnorm(const float* o, const void* z, bool z_f32, const float* weight,

@@ -1,6 +1,6 @@
-// tma_map.h -- host-side construction of the TMA tensor maps used by the tensor-core
-// prefill: 2-D bf16 views [rows, width] read in boxes of 64 elements x 32 rows with the
-// 128-byte swizzle (one box row = one 128-byte swizzle row).
+// tma_map.h -- host-side construction of 2-D bf16 TMA tensor maps [rows, width]: the
+// tensor-core prefill's (boxes of 64 elements x 32 rows with the 128-byte swizzle, one box
+// row = one 128-byte swizzle row) and plain row-major boxes for streaming passes.
 #pragma once
 
 #include <cuda.h>
@@ -33,6 +33,22 @@ inline bool make_bf16_map(CUtensorMap* map, const void* base, uint64_t width, ui
     const cuuint32_t estr[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// Row pitch = width elements (16-byte multiple); boxes of box_w x box_h elements stored
+// row-major without swizzle; rows and columns outside the tensor read as zero.
+inline bool make_bf16_map_plain(CUtensorMap* map, const void* base, uint64_t width,
+                                uint64_t rows, uint32_t box_w, uint32_t box_h) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {width, rows};
+    const cuuint64_t strides[1] = {width * 2};
+    const cuuint32_t box[2] = {box_w, box_h};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }

@@ -78,8 +78,9 @@ cudaError_t launch_prefill_tc(const FwdParams& p, cudaStream_t stream) {
 int read_and_clear_tc_status() {
     const int v64 = read_and_clear_tc64_status();
     const int vst = read_and_clear_selftest_status();
-    if (v64 < 0 || vst < 0) return -1;
-    return v64 != 0 ? v64 : vst;
+    const int vcv = read_and_clear_conv_status();
+    if (v64 < 0 || vst < 0 || vcv < 0) return -1;
+    return v64 != 0 ? v64 : vst != 0 ? vst : vcv;
 }
 
 }  // namespace gdr

@@ -328,7 +328,8 @@ GDR_API int gdr_gated_rmsnorm_f32(const float* o, const float* z, const float* w
 
 /*
  * Device-side status of the kernels enqueued so far.  Synchronises `stream`, then returns
- * GDR_ERR_TIMEOUT if any tensor-core prefill kernel abandoned one of its bounded waits
+ * GDR_ERR_TIMEOUT if any tensor-core prefill kernel (or the TMA-fed convolution that
+ * gdr_short_conv_silu runs for T >= 256) abandoned one of its bounded waits
  * (each wait on an mbarrier gives up after 2 s, records the event and lets the kernel
  * exit instead of hanging), GDR_ERR_CUDA if the stream reports an error, else GDR_OK.
  * The timeout record is cleared by the call.
