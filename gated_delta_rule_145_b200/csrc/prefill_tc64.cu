@@ -319,11 +319,16 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float gj[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < 8; e += 2) {
                 const int jj = 8 * kc + e;
                 // e^{G_i - G_j} r_k,j = 2^{G2_i - G2r_j}
-                const float pv = f * ex2_approx(Gi2 - gj[e]) * v[e];
-                p[e] = (jj < i || (!arow && jj == i)) ? pv : 0.f;
+                const float2 d = __ffma2_rn(make_float2(gj[e], gj[e + 1]), make_float2(-1.f, -1.f),
+                                            make_float2(Gi2, Gi2));
+                const float2 ex = make_float2(ex2_approx(d.x), ex2_approx(d.y));
+                const float2 pv = __fmul2_rn(__fmul2_rn(make_float2(f, f), ex),
+                                             make_float2(v[e], v[e + 1]));
+                p[e] = (jj < i || (!arow && jj == i)) ? pv.x : 0.f;
+                p[e + 1] = (jj + 1 < i || (!arow && jj + 1 == i)) ? pv.y : 0.f;
             }
             if (arow) {
                 *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc]) = make_float4(p[0], p[1], p[2], p[3]);
@@ -363,8 +368,10 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int m = 0; m < (i & ~1); m += 2) {
                 const float2 av = *reinterpret_cast<const float2*>(&sm.w.Am[o + i][o + m]);
-                s0 -= av.x * x[m];
-                s1 -= av.y * x[m + 1];
+                const float2 ss = __ffma2_rn(make_float2(-av.x, -av.y), make_float2(x[m], x[m + 1]),
+                                             make_float2(s0, s1));
+                s0 = ss.x;
+                s1 = ss.y;
             }
             if (i & 1) s0 -= sm.w.Am[o + i][o + i - 1] * x[i - 1];
             x[i] = s0 + s1;
@@ -390,7 +397,9 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int m = 0; m < 16; ++m) {
             const float a_ = sm.w.Am[o + 16 + i][o + m];
             const float4 t4 = *reinterpret_cast<const float4*>(&sm.w.Tm[o + m][o + jc]);
-            z[0] += a_ * t4.x; z[1] += a_ * t4.y; z[2] += a_ * t4.z; z[3] += a_ * t4.w;
+            const float2 z01 = __ffma2_rn(make_float2(a_, a_), make_float2(t4.x, t4.y), make_float2(z[0], z[1]));
+            const float2 z23 = __ffma2_rn(make_float2(a_, a_), make_float2(t4.z, t4.w), make_float2(z[2], z[3]));
+            z[0] = z01.x; z[1] = z01.y; z[2] = z23.x; z[3] = z23.y;
         }
         *reinterpret_cast<float4*>(&sm.w.Am[o + i][o + jc]) = make_float4(z[0], z[1], z[2], z[3]);
     }
@@ -406,7 +415,9 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int m = 0; m < mend; ++m) {
             const float tv = sm.w.Tm[o + 16 + i][o + 16 + m];
             const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Am[o + m][o + jc]);
-            t[0] += tv * z4.x; t[1] += tv * z4.y; t[2] += tv * z4.z; t[3] += tv * z4.w;
+            const float2 t01 = __ffma2_rn(make_float2(tv, tv), make_float2(z4.x, z4.y), make_float2(t[0], t[1]));
+            const float2 t23 = __ffma2_rn(make_float2(tv, tv), make_float2(z4.z, z4.w), make_float2(t[2], t[3]));
+            t[0] = t01.x; t[1] = t01.y; t[2] = t23.x; t[3] = t23.y;
         }
         *reinterpret_cast<float4*>(&sm.w.Tm[o + 16 + i][o + jc]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
     }
@@ -425,8 +436,13 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float a_ = sm.w.Am[m][32 + i];
             const float4 t0v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0]);
             const float4 t1v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0 + 4]);
-            z[0] += a_ * t0v.x; z[1] += a_ * t0v.y; z[2] += a_ * t0v.z; z[3] += a_ * t0v.w;
-            z[4] += a_ * t1v.x; z[5] += a_ * t1v.y; z[6] += a_ * t1v.z; z[7] += a_ * t1v.w;
+            const float2 a2 = make_float2(a_, a_);
+            const float2 za = __ffma2_rn(a2, make_float2(t0v.x, t0v.y), make_float2(z[0], z[1]));
+            const float2 zb = __ffma2_rn(a2, make_float2(t0v.z, t0v.w), make_float2(z[2], z[3]));
+            const float2 zc = __ffma2_rn(a2, make_float2(t1v.x, t1v.y), make_float2(z[4], z[5]));
+            const float2 zd = __ffma2_rn(a2, make_float2(t1v.z, t1v.w), make_float2(z[6], z[7]));
+            z[0] = za.x; z[1] = za.y; z[2] = zb.x; z[3] = zb.y;
+            z[4] = zc.x; z[5] = zc.y; z[6] = zd.x; z[7] = zd.y;
         }
         *reinterpret_cast<float4*>(&sm.w.Am[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
         *reinterpret_cast<float4*>(&sm.w.Am[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
@@ -444,8 +460,13 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float tv = sm.w.Tm[32 + i][32 + m];
             const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0]);
             const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0 + 4]);
-            t[0] += tv * z0.x; t[1] += tv * z0.y; t[2] += tv * z0.z; t[3] += tv * z0.w;
-            t[4] += tv * z1.x; t[5] += tv * z1.y; t[6] += tv * z1.z; t[7] += tv * z1.w;
+            const float2 t2 = make_float2(tv, tv);
+            const float2 ta = __ffma2_rn(t2, make_float2(z0.x, z0.y), make_float2(t[0], t[1]));
+            const float2 tb = __ffma2_rn(t2, make_float2(z0.z, z0.w), make_float2(t[2], t[3]));
+            const float2 tc_ = __ffma2_rn(t2, make_float2(z1.x, z1.y), make_float2(t[4], t[5]));
+            const float2 td = __ffma2_rn(t2, make_float2(z1.z, z1.w), make_float2(t[6], t[7]));
+            t[0] = ta.x; t[1] = ta.y; t[2] = tb.x; t[3] = tb.y;
+            t[4] = tc_.x; t[5] = tc_.y; t[6] = td.x; t[7] = td.y;
         }
         *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
         *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0 + 4]) = make_float4(-t[4], -t[5], -t[6], -t[7]);
@@ -598,18 +619,24 @@ __device__ __forceinline__ void put16s(uint8_t* op, uint32_t lo_off, int k, int 
 }
 
 // v = (sc * v + hi) + lo over 16 columns of a [hi | lo] accumulator from taddr (both
-// loads in flight before one wait).
+// loads in flight before one wait), on paired fp32 instructions.
 __device__ __forceinline__ void ld_acc16s(uint32_t taddr, float sc, float (&v)[16]) {
     float hi[16], lo[16];
     tmem_ld16(taddr, hi);
     tmem_ld16(taddr + NT, lo);
     tmem_ld_wait();
+    const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = (sc * v[i] + hi[i]) + lo[i];
+    for (int i = 0; i < 16; i += 2) {
+        const float2 t = __ffma2_rn(sc2, make_float2(v[i], v[i + 1]), make_float2(hi[i], hi[i + 1]));
+        const float2 u = __fadd2_rn(t, make_float2(lo[i], lo[i + 1]));
+        v[i] = u.x;
+        v[i + 1] = u.y;
+    }
 }
 
 // v = (sc * v + hi) + lo over 24 columns of a [hi | lo] accumulator from taddr (all four
-// loads in flight before one wait).
+// loads in flight before one wait), on paired fp32 instructions.
 __device__ __forceinline__ void ld_acc24s(uint32_t taddr, float sc, float (&v)[24]) {
     float hi[24], lo[24];
     tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&hi[0]));
@@ -617,8 +644,14 @@ __device__ __forceinline__ void ld_acc24s(uint32_t taddr, float sc, float (&v)[2
     tmem_ld16(taddr + NT, *reinterpret_cast<float(*)[16]>(&lo[0]));
     tmem_ld8(taddr + NT + 16, &lo[16]);
     tmem_ld_wait();
+    const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-    for (int i = 0; i < 24; ++i) v[i] = (sc * v[i] + hi[i]) + lo[i];
+    for (int i = 0; i < 24; i += 2) {
+        const float2 t = __ffma2_rn(sc2, make_float2(v[i], v[i + 1]), make_float2(hi[i], hi[i + 1]));
+        const float2 u = __fadd2_rn(t, make_float2(lo[i], lo[i + 1]));
+        v[i] = u.x;
+        v[i + 1] = u.y;
+    }
 }
 
 struct Sp64Ctx {
@@ -888,8 +921,11 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 fv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[e]));
-                v[8 * g + 2 * e] = bet * fv.x - wv * v[8 * g + 2 * e];
-                v[8 * g + 2 * e + 1] = bet * fv.y - wv * v[8 * g + 2 * e + 1];
+                const float2 t = __fmul2_rn(make_float2(-wv, -wv),
+                                            make_float2(v[8 * g + 2 * e], v[8 * g + 2 * e + 1]));
+                const float2 u = __ffma2_rn(make_float2(bet, bet), fv, t);
+                v[8 * g + 2 * e] = u.x;
+                v[8 * g + 2 * e + 1] = u.y;
             }
         }
         put16s(sm.b_op, OPB, r, 2 * ct, C64, v, 1.f);
