@@ -302,7 +302,9 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ---- A rows into shared memory (warps 0, 1); P rows straight into the record's
     //      image rows 64-127 (warps 2, 3).  Accumulator row 32 w + lane (warps 0, 1: K K^T,
     //      2, 3: Q K^T), read eight columns at a time.
-    {
+    // erase = 0 (gated linear attention): A = 0, so T = I, which the state kernel's erase =
+    // 0 instance never reads: only the P rows (warps 2, 3) and the vectors are written
+    if (erase || warp >= 2) {
         const bool arow = warp < 2;
         const int i = 32 * (warp & 1) + lane;
         const float Gi2 = sm.G2[i];
@@ -355,139 +357,140 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 64);
-
-    // ---- T = (I + A)^-1.  The four diagonal 16 x 16 blocks by forward substitution, one
-    //      column per lane (warps 0 and 1: lanes 0-15 and 16-31 take one block each);
-    //      warps 2 and 3 zero the blocks above the diagonal.
-    if (warp < 2) {
-        const int o = 32 * warp + (lane & 16), j = lane & 15;
-        float x[16];
+    if (erase) {
+        // ---- T = (I + A)^-1.  The four diagonal 16 x 16 blocks by forward substitution, one
+        //      column per lane (warps 0 and 1: lanes 0-15 and 16-31 take one block each);
+        //      warps 2 and 3 zero the blocks above the diagonal.
+        if (warp < 2) {
+            const int o = 32 * warp + (lane & 16), j = lane & 15;
+            float x[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float s0 = i == j ? 1.f : 0.f, s1 = 0.f;
+            for (int i = 0; i < 16; ++i) {
+                float s0 = i == j ? 1.f : 0.f, s1 = 0.f;
 #pragma unroll
-            for (int m = 0; m < (i & ~1); m += 2) {
-                const float2 av = *reinterpret_cast<const float2*>(&sm.w.Am[o + i][o + m]);
-                const float2 ss = __ffma2_rn(make_float2(-av.x, -av.y), make_float2(x[m], x[m + 1]),
-                                             make_float2(s0, s1));
-                s0 = ss.x;
-                s1 = ss.y;
+                for (int m = 0; m < (i & ~1); m += 2) {
+                    const float2 av = *reinterpret_cast<const float2*>(&sm.w.Am[o + i][o + m]);
+                    const float2 ss = __ffma2_rn(make_float2(-av.x, -av.y), make_float2(x[m], x[m + 1]),
+                                                 make_float2(s0, s1));
+                    s0 = ss.x;
+                    s1 = ss.y;
+                }
+                if (i & 1) s0 -= sm.w.Am[o + i][o + i - 1] * x[i - 1];
+                x[i] = s0 + s1;
             }
-            if (i & 1) s0 -= sm.w.Am[o + i][o + i - 1] * x[i - 1];
-            x[i] = s0 + s1;
-        }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sm.w.Tm[o + i][o + j] = x[i];
-    } else {
-        // the zero blocks above the diagonal inside each 32-token block, (0,1) and (2,3),
-        // which the 32-level coupling reads (the upper-right 32 x 32 block of the image is
-        // written as zeros directly)
-        for (int e = tid - 64; e < 2 * 256; e += 64) {
-            const int blk = e >> 8, w = e & 255, r = w >> 4, cc = w & 15;
-            sm.w.Tm[32 * blk + r][32 * blk + 16 + cc] = 0.f;
-        }
-    }
-    __syncthreads();
-    {
-        // 16-level coupling inside each 32-token block (its triangular solve):
-        // Z = A[b+16.., b..] T[b.., b..], thread -> (block bi, row i, 4 columns)
-        const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
-        float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float a_ = sm.w.Am[o + 16 + i][o + m];
-            const float4 t4 = *reinterpret_cast<const float4*>(&sm.w.Tm[o + m][o + jc]);
-            const float2 z01 = __ffma2_rn(make_float2(a_, a_), make_float2(t4.x, t4.y), make_float2(z[0], z[1]));
-            const float2 z23 = __ffma2_rn(make_float2(a_, a_), make_float2(t4.z, t4.w), make_float2(z[2], z[3]));
-            z[0] = z01.x; z[1] = z01.y; z[2] = z23.x; z[3] = z23.y;
-        }
-        *reinterpret_cast<float4*>(&sm.w.Am[o + i][o + jc]) = make_float4(z[0], z[1], z[2], z[3]);
-    }
-    __syncthreads();
-    {
-        // T[b+16.., b..] = -T[b+16.., b+16..] Z.  That block is lower triangular: row i needs
-        // m <= i only; a warp's rows end at 7 or 15, and the zero upper triangle it still
-        // reads below that is stored.
-        const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
-        const int mend = (warp & 1) ? 16 : 8;
-        float t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int m = 0; m < mend; ++m) {
-            const float tv = sm.w.Tm[o + 16 + i][o + 16 + m];
-            const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Am[o + m][o + jc]);
-            const float2 t01 = __ffma2_rn(make_float2(tv, tv), make_float2(z4.x, z4.y), make_float2(t[0], t[1]));
-            const float2 t23 = __ffma2_rn(make_float2(tv, tv), make_float2(z4.z, z4.w), make_float2(t[2], t[3]));
-            t[0] = t01.x; t[1] = t01.y; t[2] = t23.x; t[3] = t23.y;
-        }
-        *reinterpret_cast<float4*>(&sm.w.Tm[o + 16 + i][o + jc]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
-    }
-    __syncthreads();
-    {
-        // 32-level coupling: Z = A_ba T_a (rows 32-63, columns 0-31), warp w -> columns
-        // 8 w .. 8 w + 7, lane -> row.  T_a is lower triangular: column j needs m >= j, so
-        // the warp starts at m = 8 w (the zeros it reads above the diagonal are stored);
-        // A_ba comes from its transposed copy (consecutive lanes, consecutive words).
-        const int i = lane, j0 = 8 * warp;
-        float z[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) z[q] = 0.f;
-#pragma unroll 4
-        for (int m = j0; m < 32; ++m) {
-            const float a_ = sm.w.Am[m][32 + i];
-            const float4 t0v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0]);
-            const float4 t1v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0 + 4]);
-            const float2 a2 = make_float2(a_, a_);
-            const float2 za = __ffma2_rn(a2, make_float2(t0v.x, t0v.y), make_float2(z[0], z[1]));
-            const float2 zb = __ffma2_rn(a2, make_float2(t0v.z, t0v.w), make_float2(z[2], z[3]));
-            const float2 zc = __ffma2_rn(a2, make_float2(t1v.x, t1v.y), make_float2(z[4], z[5]));
-            const float2 zd = __ffma2_rn(a2, make_float2(t1v.z, t1v.w), make_float2(z[6], z[7]));
-            z[0] = za.x; z[1] = za.y; z[2] = zb.x; z[3] = zb.y;
-            z[4] = zc.x; z[5] = zc.y; z[6] = zd.x; z[7] = zd.y;
-        }
-        *reinterpret_cast<float4*>(&sm.w.Am[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
-        *reinterpret_cast<float4*>(&sm.w.Am[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
-    }
-    __syncthreads();
-    {
-        // T_ba = -T_b Z.  T_b is lower triangular: row i needs m <= i only; warp w holds rows
-        // 8 w .. 8 w + 7 (the zero upper triangle it reads below 8 w + 8 is stored).
-        const int i = tid >> 2, j0 = 8 * (tid & 3);
-        float t[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) t[q] = 0.f;
-#pragma unroll 4
-        for (int m = 0; m < 8 * warp + 8; ++m) {
-            const float tv = sm.w.Tm[32 + i][32 + m];
-            const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0]);
-            const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0 + 4]);
-            const float2 t2 = make_float2(tv, tv);
-            const float2 ta = __ffma2_rn(t2, make_float2(z0.x, z0.y), make_float2(t[0], t[1]));
-            const float2 tb = __ffma2_rn(t2, make_float2(z0.z, z0.w), make_float2(t[2], t[3]));
-            const float2 tc_ = __ffma2_rn(t2, make_float2(z1.x, z1.y), make_float2(t[4], t[5]));
-            const float2 td = __ffma2_rn(t2, make_float2(z1.z, z1.w), make_float2(t[6], t[7]));
-            t[0] = ta.x; t[1] = ta.y; t[2] = tb.x; t[3] = tb.y;
-            t[4] = tc_.x; t[5] = tc_.y; t[6] = td.x; t[7] = td.y;
-        }
-        *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
-        *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0 + 4]) = make_float4(-t[4], -t[5], -t[6], -t[7]);
-    }
-    __syncthreads();
-    // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread); rows 0-31 x
-    //      columns 32-63 are zero.  Eight consecutive lanes take the eight rows of one
-    //      8-row group at one chunk: one 128-byte line of the image.
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int task = tid + PREP64_THREADS * e;
-        const int row = 8 * (task >> 6) + (task & 7), kc = (task >> 3) & 7;
-        if (row < 32 && kc >= 4) {
-            const uint32_t off = r64::k_off(row, kc);
-            *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < 16; ++i) sm.w.Tm[o + i][o + j] = x[i];
         } else {
-            store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(row, kc),
-                        &sm.w.Tm[row][8 * kc], -1.f);
+            // the zero blocks above the diagonal inside each 32-token block, (0,1) and (2,3),
+            // which the 32-level coupling reads (the upper-right 32 x 32 block of the image is
+            // written as zeros directly)
+            for (int e = tid - 64; e < 2 * 256; e += 64) {
+                const int blk = e >> 8, w = e & 255, r = w >> 4, cc = w & 15;
+                sm.w.Tm[32 * blk + r][32 * blk + 16 + cc] = 0.f;
+            }
         }
-    }
+        __syncthreads();
+        {
+            // 16-level coupling inside each 32-token block (its triangular solve):
+            // Z = A[b+16.., b..] T[b.., b..], thread -> (block bi, row i, 4 columns)
+            const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
+            float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float a_ = sm.w.Am[o + 16 + i][o + m];
+                const float4 t4 = *reinterpret_cast<const float4*>(&sm.w.Tm[o + m][o + jc]);
+                const float2 z01 = __ffma2_rn(make_float2(a_, a_), make_float2(t4.x, t4.y), make_float2(z[0], z[1]));
+                const float2 z23 = __ffma2_rn(make_float2(a_, a_), make_float2(t4.z, t4.w), make_float2(z[2], z[3]));
+                z[0] = z01.x; z[1] = z01.y; z[2] = z23.x; z[3] = z23.y;
+            }
+            *reinterpret_cast<float4*>(&sm.w.Am[o + i][o + jc]) = make_float4(z[0], z[1], z[2], z[3]);
+        }
+        __syncthreads();
+        {
+            // T[b+16.., b..] = -T[b+16.., b+16..] Z.  That block is lower triangular: row i needs
+            // m <= i only; a warp's rows end at 7 or 15, and the zero upper triangle it still
+            // reads below that is stored.
+            const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
+            const int mend = (warp & 1) ? 16 : 8;
+            float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+            for (int m = 0; m < mend; ++m) {
+                const float tv = sm.w.Tm[o + 16 + i][o + 16 + m];
+                const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Am[o + m][o + jc]);
+                const float2 t01 = __ffma2_rn(make_float2(tv, tv), make_float2(z4.x, z4.y), make_float2(t[0], t[1]));
+                const float2 t23 = __ffma2_rn(make_float2(tv, tv), make_float2(z4.z, z4.w), make_float2(t[2], t[3]));
+                t[0] = t01.x; t[1] = t01.y; t[2] = t23.x; t[3] = t23.y;
+            }
+            *reinterpret_cast<float4*>(&sm.w.Tm[o + 16 + i][o + jc]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+        }
+        __syncthreads();
+        {
+            // 32-level coupling: Z = A_ba T_a (rows 32-63, columns 0-31), warp w -> columns
+            // 8 w .. 8 w + 7, lane -> row.  T_a is lower triangular: column j needs m >= j, so
+            // the warp starts at m = 8 w (the zeros it reads above the diagonal are stored);
+            // A_ba comes from its transposed copy (consecutive lanes, consecutive words).
+            const int i = lane, j0 = 8 * warp;
+            float z[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) z[q] = 0.f;
+#pragma unroll 4
+            for (int m = j0; m < 32; ++m) {
+                const float a_ = sm.w.Am[m][32 + i];
+                const float4 t0v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0]);
+                const float4 t1v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0 + 4]);
+                const float2 a2 = make_float2(a_, a_);
+                const float2 za = __ffma2_rn(a2, make_float2(t0v.x, t0v.y), make_float2(z[0], z[1]));
+                const float2 zb = __ffma2_rn(a2, make_float2(t0v.z, t0v.w), make_float2(z[2], z[3]));
+                const float2 zc = __ffma2_rn(a2, make_float2(t1v.x, t1v.y), make_float2(z[4], z[5]));
+                const float2 zd = __ffma2_rn(a2, make_float2(t1v.z, t1v.w), make_float2(z[6], z[7]));
+                z[0] = za.x; z[1] = za.y; z[2] = zb.x; z[3] = zb.y;
+                z[4] = zc.x; z[5] = zc.y; z[6] = zd.x; z[7] = zd.y;
+            }
+            *reinterpret_cast<float4*>(&sm.w.Am[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
+            *reinterpret_cast<float4*>(&sm.w.Am[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
+        }
+        __syncthreads();
+        {
+            // T_ba = -T_b Z.  T_b is lower triangular: row i needs m <= i only; warp w holds rows
+            // 8 w .. 8 w + 7 (the zero upper triangle it reads below 8 w + 8 is stored).
+            const int i = tid >> 2, j0 = 8 * (tid & 3);
+            float t[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) t[q] = 0.f;
+#pragma unroll 4
+            for (int m = 0; m < 8 * warp + 8; ++m) {
+                const float tv = sm.w.Tm[32 + i][32 + m];
+                const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0]);
+                const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0 + 4]);
+                const float2 t2 = make_float2(tv, tv);
+                const float2 ta = __ffma2_rn(t2, make_float2(z0.x, z0.y), make_float2(t[0], t[1]));
+                const float2 tb = __ffma2_rn(t2, make_float2(z0.z, z0.w), make_float2(t[2], t[3]));
+                const float2 tc_ = __ffma2_rn(t2, make_float2(z1.x, z1.y), make_float2(t[4], t[5]));
+                const float2 td = __ffma2_rn(t2, make_float2(z1.z, z1.w), make_float2(t[6], t[7]));
+                t[0] = ta.x; t[1] = ta.y; t[2] = tb.x; t[3] = tb.y;
+                t[4] = tc_.x; t[5] = tc_.y; t[6] = td.x; t[7] = td.y;
+            }
+            *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+            *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0 + 4]) = make_float4(-t[4], -t[5], -t[6], -t[7]);
+        }
+        __syncthreads();
+        // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread); rows 0-31 x
+        //      columns 32-63 are zero.  Eight consecutive lanes take the eight rows of one
+        //      8-row group at one chunk: one 128-byte line of the image.
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int task = tid + PREP64_THREADS * e;
+            const int row = 8 * (task >> 6) + (task & 7), kc = (task >> 3) & 7;
+            if (row < 32 && kc >= 4) {
+                const uint32_t off = r64::k_off(row, kc);
+                *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
+            } else {
+                store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(row, kc),
+                            &sm.w.Tm[row][8 * kc], -1.f);
+            }
+        }
+    }  // erase
     // ---- vectors
     if (tid < C64) {
         const int i = tid;
@@ -659,6 +662,7 @@ struct Sp64Ctx {
     int v_zero;         // v = 0: B = -diag(w) K S (the segment map Phi)
     int init_identity;  // S_0 = I (the segment map Phi) instead of init_state or zeros
     bool has_out;       // outputs wanted (else no P Delta product and no output epilogue)
+    bool gla;           // erase = 0: Delta = B = diag(beta) V, only the P rows of the record
     long long t0, t1, rbase;
     const uint8_t* ws;
     uint32_t tmem;
@@ -678,7 +682,9 @@ __device__ void issue_loads(Sp64Smem& sm, const Sp64Ctx& x, int s, const CUtenso
                             const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
     const int r = s & 1;
     uint64_t* bar = &sm.full[r];
-    mbar_arrive_expect_tx(bar, (x.v_zero ? 8u : 10u) * 4096u + 2u * r64::PART + r64::VEC_BYTES);
+    // erase = 0: the record's -T rows (0-63) are neither written nor read
+    const uint32_t part = x.gla ? r64::PART / 2 : r64::PART;
+    mbar_arrive_expect_tx(bar, (x.v_zero ? 8u : 10u) * 4096u + 2u * part + r64::VEC_BYTES);
     const int y = (int)(x.t0 + (long long)s * C64);
 #pragma unroll 1
     for (int hf = 0; hf < 2; ++hf) {
@@ -694,8 +700,9 @@ __device__ void issue_loads(Sp64Smem& sm, const Sp64Ctx& x, int s, const CUtenso
         tma_load_2d(sm.vt[r] + 4096, tm_v, x.h * DV + x.col0, y + 32, bar);
     }
     const uint8_t* rc = x.record(s);
-    bulk_load(sm.rec[r], rc + r64::OFF_A, r64::PART, bar);
-    bulk_load(sm.rec[r] + r64::PART, rc + r64::OFF_A + r64::PART, r64::PART, bar);
+    const uint32_t skip = r64::PART - part;  // rows 0-63 are the first half of a part
+    bulk_load(sm.rec[r] + skip, rc + r64::OFF_A + skip, part, bar);
+    bulk_load(sm.rec[r] + r64::PART + skip, rc + r64::OFF_A + r64::PART + skip, part, bar);
     bulk_load(sm.vec[r], rc + r64::OFF_VEC, r64::VEC_BYTES, bar);
 }
 
@@ -732,8 +739,9 @@ __device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane, const CU
                 mma_commit(&sm.empty[r]);
                 if (s >= 1) mbar_arrive(&sm.g1_issued);
             }
-            // block s + 1 into slot (s + 1) & 1, once block s - 1 is done with it
-            if (live && s >= 1 && s + 1 < x.n) {
+            // block s + 1 into slot (s + 1) & 1, once block s - 1 is done with it (erase = 0:
+            // the BD group's first warp issues them, as early as the slot frees)
+            if (!x.gla && live && s >= 1 && s + 1 < x.n) {
                 live = w64(ab, &sm.empty[(s + 1) & 1], (uint32_t)((s - 1) >> 1) & 1u);
                 if (live) {
                     issue_loads(sm, x, s + 1, tm_q, tm_k, tm_v);
@@ -746,15 +754,19 @@ __device__ void g1_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane, const CU
     if (leader) {
         mma_commit(&sm.drain_s);
         mbar_wait(&sm.drain_s, 0);
-        // every copy this warp started has landed before the CTA may exit
-        for (int s = max(0, armed - 1); s <= armed; ++s)
-            mbar_wait(&sm.full[s & 1], (uint32_t)(s >> 1) & 1u);
+        // every copy this warp started has landed before the CTA may exit (erase = 0: the
+        // BD group, which issued all loads after the first two, waits for its own)
+        if (!x.gla)
+            for (int s = max(0, armed - 1); s <= armed; ++s)
+                mbar_wait(&sm.full[s & 1], (uint32_t)(s >> 1) & 1u);
     }
     __syncwarp();
 }
 
 // Warp 18: Delta(s) = [-T; P] [B hi | lo] into acc2; G3(s) = K_s^T [D Delta hi | lo] into
-// acc3; [-T; P] [Delta hi | lo] into acc4.
+// acc3; [-T; P] [Delta hi | lo] into acc4.  kGla (erase = 0, T = I): no Delta product; G3
+// and P Delta on the operands the BD group writes straight from V, one barrier per block.
+template <bool kGla>
 __device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
     const uint32_t id96 = idesc_bf16(128, 2 * NT, 0, 1);
     const uint32_t id48 = idesc_bf16(128, NT, 0, 1);
@@ -778,7 +790,31 @@ __device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
                      dadd64(dx, ks * 256), id48, 1);
     };
     bool live = true;
-    for (int s = 0; s < x.n; ++s) {
+    if (kGla) {
+        for (int s = 0; s < x.n; ++s) {
+            const int r = s & 1;
+            if (leader && live)
+                live = w64(ab, &sm.full[r], (uint32_t)(s >> 1) & 1u) &&
+                       (s < 1 || w64(ab, &sm.acc3_free, (uint32_t)(s - 1) & 1u)) &&
+                       (s < 1 || !x.has_out || w64(ab, &sm.acc4_free, (uint32_t)(s - 1) & 1u));
+            gbar(BAR_BD, BAR_BD_THREADS);  // D Delta_s and Delta_s written
+            if (leader && live) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(x.tmem + T_ACC3, dadd64(d_kt, r * 32768 + ks * 2048),
+                             dadd64(d_dd, ks * 256), id_g3, ks > 0);
+                mma_commit(&sm.acc3_full);
+                if (x.has_out) {
+                    tp_product(r, T_ACC4, d_d);
+                    mma_commit(&sm.acc4_full);
+                }
+                mma_commit(&sm.empty[r]);
+            }
+            __syncwarp();
+        }
+    }
+    for (int s = 0; s < (kGla ? 0 : x.n); ++s) {
         const int r = s & 1;
         if (leader && live) live = w64(ab, &sm.full[r], (uint32_t)(s >> 1) & 1u);
         gbar(BAR_BD, BAR_BD_THREADS);  // B_s written
@@ -878,8 +914,12 @@ __device__ void s64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
 
 // ---------------------------------------- BD group (warps 8, 9, 12, 13, 16, 17)
 // Warp w: accumulator rows 32 (w % 4) + lane (tokens 0-63), columns 16 ct .. 16 ct + 15 with
-// ct = (w - 8) / 4.
-__device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
+// ct = (w - 8) / 4.  kGla (erase = 0): B = diag(beta) V is Delta itself; D Delta and Delta
+// are written from V without waiting for K S, so this group runs ahead of the state.
+template <bool kGla>
+__device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
+                        const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                        const CUtensorMap* tm_v) {
     const int q = warp & 3, ct = (warp - 8) >> 2;
     const int r = 32 * q + lane;  // token of the block (accumulator rows 0-63)
     const int j0 = 16 * ct;
@@ -887,8 +927,21 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
     const int nv = DV - (x.col0 + j0);  // columns of V that exist
     int* ab = &sm.abort;
     bool live = true;
+    int armed = min(x.n, 2) - 1;  // erase = 0, warp 8: the last block whose loads were issued
     for (int s = 0; s < x.n; ++s) {
         const int rs = s & 1;
+        // erase = 0: block s + 1 into the slot block s - 1 frees (its G1 and P Delta), which
+        // needs nothing from this group, so the operands stay a block ahead of the state
+        if (kGla && warp == 8 && s >= 1 && s + 1 < x.n) {
+            if (lane == 0 && live) {
+                live = w64(ab, &sm.empty[(s + 1) & 1], (uint32_t)((s - 1) >> 1) & 1u);
+                if (live) {
+                    issue_loads(sm, x, s + 1, tm_q, tm_k, tm_v);
+                    armed = s + 1;
+                }
+            }
+            live = __shfl_sync(0xffffffffu, live, 0);
+        }
         live = live && w64(ab, &sm.full[rs], (uint32_t)(s >> 1) & 1u);
         const float bet = sm.vec[rs][r64::VEC_BETA + r], wv = sm.vec[rs][r64::VEC_W + r];
         const float d = sm.vec[rs][r64::VEC_D + r];
@@ -906,15 +959,17 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
                         : make_uint4(0, 0, 0, 0);
         }
         // B = beta V - w K S
-        live = live && w64(ab, &sm.acc1_full[s & 1], (uint32_t)(s >> 1) & 1u);
         float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.f;
-        if (live) {
-            tc_fence_after();
-            ld_acc16s(tl + T_ACC1 + 96 * (s & 1) + j0, 0.f, v);
+        if (!kGla) {
+            live = live && w64(ab, &sm.acc1_full[s & 1], (uint32_t)(s >> 1) & 1u);
+            if (live) {
+                tc_fence_after();
+                ld_acc16s(tl + T_ACC1 + 96 * (s & 1) + j0, 0.f, v);
+            }
+            warp_arrive64(&sm.acc1_free[s & 1], lane);
         }
-        warp_arrive64(&sm.acc1_free[s & 1], lane);
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
             const uint32_t wd[4] = {vc[g].x, vc[g].y, vc[g].z, vc[g].w};
@@ -927,6 +982,21 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
                 v[8 * g + 2 * e] = u.x;
                 v[8 * g + 2 * e + 1] = u.y;
             }
+        }
+        if (kGla) {
+            // the operands of block s replace those of s - 1 once G3(s - 1) and P Delta(s - 1)
+            // have read them (neither can have run past block s - 1: both need these)
+            live = live && (s < 1 || (w64(ab, &sm.acc3_full, (uint32_t)(s - 1) & 1u) &&
+                                      (!x.has_out ||
+                                       w64(ab, &sm.acc4_full, (uint32_t)(s - 1) & 1u))));
+            if (live) {
+                tc_fence_after();
+                put16s(sm.dd_op, OPB, r, 2 * ct, C64, v, d);
+                if (x.has_out) put16s(sm.d_op, OPB, r, 2 * ct, C64, v, 1.f);
+                fence_async_smem();
+            }
+            gbar(BAR_BD, BAR_BD_THREADS);  // D Delta_s and Delta_s written: G3(s), P Delta(s)
+            continue;
         }
         put16s(sm.b_op, OPB, r, 2 * ct, C64, v, 1.f);
         fence_async_smem();
@@ -947,6 +1017,12 @@ __device__ void bd_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane) {
         }
         gbar(BAR_BD, BAR_BD_THREADS);  // Delta_s written: P Delta(s)
     }
+    // every copy this warp started has landed before the CTA may exit (waits on the last
+    // phase of each slot: both are complete once the blocks were consumed)
+    if (kGla && warp == 8 && lane == 0)
+        for (int s = max(0, armed - 1); s <= armed; ++s)
+            mbar_wait(&sm.full[s & 1], (uint32_t)(s >> 1) & 1u);
+    __syncwarp();
 }
 
 // ---------------------------------------------- output group (warps 10, 11, 14, 15)
@@ -1000,8 +1076,10 @@ __device__ void o64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
 }
 
 // kMap: the segment-map instance (flags at run time, gridDim.y = 2 runs N and Phi
-// together); the prefill instance has them fixed (v, outputs, init_state or zeros).
-template <bool kMap>
+// together); the prefill instances have them fixed (v, outputs, init_state or zeros).
+// kGla: the erase = 0 form (gated linear attention), whose Delta = diag(beta) V does not
+// wait for the state.
+template <bool kMap, bool kGla>
 __global__ void __launch_bounds__(SP_THREADS, 1)
 state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v,
@@ -1036,6 +1114,7 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     x.v_zero = v_zero;
     x.init_identity = init_identity;
     x.has_out = !kMap || out != nullptr;
+    x.gla = kGla;
     const int ncols = min(NT, DV - x.col0);
     if (x.n == 0) {  // empty sequence: the final state is the initial one
         grid_dep_wait();
@@ -1063,7 +1142,7 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], 2);      // G1 and the last P Delta product of the block
             mbar_init(&sm.acc1_full[i], 1);
-            mbar_init(&sm.acc1_free[i], 10);  // BD and output warps
+            mbar_init(&sm.acc1_free[i], kGla ? 4 : 10);  // (BD and) output warps
         }
         mbar_init(&sm.acc2_full, 1);
         mbar_init(&sm.g1_issued, 1);
@@ -1091,9 +1170,10 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp < 8)
         s64_role(sm, x, warp, lane, init_state, final_state);
     else if (warp < 18)
-        ((warp & 3) < 2) ? bd_role(sm, x, warp, lane) : o64_role(sm, x, warp, lane, out);
+        ((warp & 3) < 2) ? bd_role<kGla>(sm, x, warp, lane, &tm_q, &tm_k, &tm_v)
+                         : o64_role(sm, x, warp, lane, out);
     else if (warp == 18)
-        d_issue_role(sm, x, lane);
+        d_issue_role<kGla>(sm, x, lane);
     else
         g1_issue_role(sm, x, lane, &tm_q, &tm_k, &tm_v);
 
@@ -1138,11 +1218,14 @@ cudaError_t prepare64(const FwdParams& p, Maps64& m) {
     cudaError_t e = cudaFuncSetAttribute(intra64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(Prep64Smem));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(state64_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(Sp64Smem));
+    e = cudaFuncSetAttribute(state64_kernel<false, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Sp64Smem));
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(state64_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)sizeof(Sp64Smem));
+    e = cudaFuncSetAttribute(state64_kernel<false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Sp64Smem));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(state64_kernel<true, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Sp64Smem));
 }
 
 cudaError_t launch_intra64(const FwdParams& p, const Maps64& m, void* ws, cudaStream_t stream) {
@@ -1170,7 +1253,10 @@ cudaError_t launch_state64(const FwdParams& p, const Maps64& m, const void* ws, 
     cfg.attrs = attr;
     cfg.numAttrs = dependent ? 1 : 0;
     const bool map = phi || p.v_zero || p.init_identity || !p.out;
-    return cudaLaunchKernelEx(&cfg, map ? state64_kernel<true> : state64_kernel<false>, m.q, m.k,
+    if (!p.erase && map) return cudaErrorNotSupported;  // the maps are the rule's only
+    auto* kern = map ? state64_kernel<true, false>
+                     : (p.erase ? state64_kernel<false, false> : state64_kernel<false, true>);
+    return cudaLaunchKernelEx(&cfg, kern, m.q, m.k,
                               m.v, (const uint8_t*)ws,
                               (const float*)p.init_state, p.out, p.final_state,
                               (const int32_t*)p.cu_seqlens, p.T, p.Hk, p.Hv, p.v_zero,

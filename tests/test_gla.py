@@ -9,7 +9,7 @@ import pytest
 import gated_delta_rule_145_b200 as gdr
 from gated_delta_rule_145_b200 import synth
 
-from .helpers import TAU, assert_parity, oracle_forward, rel_max_err, to_device
+from .helpers import TAU, assert_parity, check_all_heads, oracle_forward, rel_max_err, to_device
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -89,6 +89,13 @@ def test_gla_decode_steps():
 
 
 @pytest.mark.slow
-def test_gla_full_prefill_T8192_sampled_heads():
+def test_gla_full_prefill_T8192_all_heads():
+    """the bench's GLA workload (B=1, T=8192, H=48, d=128): every head and the whole state
+    against the oracle's erase=False, with the same bound as the rule"""
     inp = synth.workload(2)
-    _check(inp, "chunked", heads=[0, 17, 47])
+    d = to_device(inp)
+    out, fin = gdr.prefill(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                           d["init_state"], d["cu_seqlens"], form="chunked", erase=False)
+    torch.cuda.synchronize()
+    assert gdr.gdr_device_status() == gdr.GDR_OK
+    check_all_heads(inp, _np(out), _np(fin), TAU[inp.dtype], "gla T=8192", erase=False)
