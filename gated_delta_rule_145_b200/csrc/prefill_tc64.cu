@@ -25,9 +25,10 @@
 // part moves the result by ~1e-2 of its RMS at the workload sizes, against a 2e-3 bound.
 //
 // Kernels:
-//   intra64_kernel  one CTA per (64-token block, value head): gates, norms, the Gram
-//                   [K; Q] K^T on tcgen05, A and P, T, and a record holding the operand
-//                   image [-T; P] (128 x 64, hi and lo) and the block's vectors.
+//   intra64_kernel  one CTA per (64-token block, key head): norms and the Gram [K; Q] K^T
+//                   on tcgen05 once, then per value head of the key head its gates, A and
+//                   P, T, and a record holding the operand image [-T; P] (128 x 64, hi and
+//                   lo) and the block's vectors.
 //   state64_kernel  one CTA per (sequence, value head, 48-column slice of dv); per block
 //                   the products G1 = [K; Q] [S hi | lo], Delta = [-T; P] [B hi | lo]
 //                   (rows 0-63: -Delta), G3 = K^T [D Delta hi | lo] and [-T; P] [Delta hi |
@@ -198,33 +199,50 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     // the state kernel may be scheduled as SMs drain; it waits for this grid's completion
     grid_dep_launch_dependents();
-    const int h = blockIdx.x % Hv;
-    const long long f = blockIdx.x / Hv;
+    // one CTA per (block, key head): the tiles, the Gram and the norms serve the key head's
+    // Hv / Hk value heads, whose gates, A, P, T and records follow one after another
+    const int grp = Hv / Hk;
+    const int kh = blockIdx.x % Hk;
+    const long long f = blockIdx.x / Hk;
     int s, c;
     if (!r64::locate(cu_seqlens, T, nseq, f, s, c)) return;  // past the last block
     long long t0, t1;
     seq_range(cu_seqlens, s, T, t0, t1);
     const long long c0 = t0 + (long long)c * C64;
     const int n = (int)min((long long)C64, t1 - c0);
-    const int kh = h / (Hv / Hk);
-    uint8_t* rc = ws + ((size_t)f * Hv + h) * r64::BYTES;
+    int h = kh * grp;
     if ((smem_u32(smem_raw) & 1023u) != 0) {  // swizzled tiles need 1 KB alignment
         if (tid == 0) atomicExch(&g_tc64_status, 2);
         return;
     }
-    // gate inputs: warp 2 tokens 0-31, warp 3 tokens 32-63 (padding rows read nothing)
+    // gate inputs of value head hh: warp 2 tokens 0-31, warp 3 tokens 32-63 (padding rows
+    // read nothing)
     __nv_bfloat16 ga{}, gb{};
     float A_lg = 0.f, dtb = 0.f;
-    if (warp >= 2) {
-        A_lg = A_log[h];
-        dtb = dt_bias[h];
-        const int i = 32 * (warp - 2) + lane;
-        if (i < n) {
-            const size_t th = (size_t)(c0 + i) * Hv + h;
-            ga = a[th];
-            gb = b[th];
+    auto load_gates = [&](int hh) {
+        if (warp >= 2) {
+            A_lg = A_log[hh];
+            dtb = dt_bias[hh];
+            const int i = 32 * (warp - 2) + lane;
+            if (i < n) {
+                const size_t th = (size_t)(c0 + i) * Hv + hh;
+                ga = a[th];
+                gb = b[th];
+            }
         }
-    }
+    };
+    // beta and the in-block cumulative G from them (warps 2, 3)
+    auto gates = [&]() {
+        if (warp >= 2) {
+            const int i = 32 * (warp - 2) + lane;
+            float g = 0.f, bt = 0.f;  // padding rows: no decay, no write
+            if (i < n)
+                gates_fast64(__bfloat162float(ga), __bfloat162float(gb), expf(A_lg), dtb, g, bt);
+            sm.beta[i] = bt;
+            sm.G[i] = scan32(g, lane);
+        }
+    };
+    load_gates(h);
     if (tid == 0) {
         mbar_init(&sm.bar_tma, 1);
         mbar_init(&sm.bar_mma, 1);
@@ -243,13 +261,7 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
-    if (warp >= 2) {
-        const int i = 32 * (warp - 2) + lane;
-        float g = 0.f, bt = 0.f;  // padding rows: no decay, no write
-        if (i < n) gates_fast64(__bfloat162float(ga), __bfloat162float(gb), expf(A_lg), dtb, g, bt);
-        sm.beta[i] = bt;
-        sm.G[i] = scan32(g, lane);
-    }
+    gates();
     bool ok = __syncthreads_and(mbar_wait(&sm.bar_tma, 0)) != 0;
     // ---- Gram [K; Q] K^T  (M = 128, N = 64, K = 128): rows 0-63 K K^T, 64-127 Q K^T
     if (warp == 0) {
@@ -268,7 +280,6 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     // ---- inverse norms of the K rows (0-63) and Q rows (64-127): a thread pair per row
     //      (the swizzle only permutes 16-byte pieces inside a row, which a sum ignores)
-    if (tid < C64) sm.G2[tid] = (sm.G[tid] + (tid >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f;
     if (ok) {
 #pragma unroll 1
         for (int e = 0; e < 2; ++e) {
@@ -278,9 +289,6 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (hf == 0) {
                 if (e == 0) {
                     sm.rk[row] = rsqrtf(ss + kNormEps);
-                    // log2(r_k) = -log2(ss + eps) / 2
-                    sm.G2r[row] = (sm.G[row] + (row >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f +
-                                  0.5f * __log2f(ss + kNormEps);
                 } else {
                     sm.rq[row - 64] = rsqrtf(ss + kNormEps) * rsqrtf((float)DK);
                 }
@@ -296,212 +304,237 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (tid == 0) atomicExch(&g_tc64_status, 1);
         return;
     }
-    const float G31 = sm.G[31];
-    auto Gf = [&](int j) { return sm.G[j] + (j >= 32 ? G31 : 0.f); };
+    for (int gi = 0; gi < grp; ++gi, ++h) {
+        uint8_t* rc = ws + ((size_t)f * Hv + h) * r64::BYTES;
+        if (gi > 0) {
+            __syncthreads();  // the previous head's last phase has read G and beta
+            gates();
+        }
+        __syncthreads();
+        // the block's G times log2(e), and with -log2(r_k): a column's decay and key scale in
+        // one exponent
+        if (tid < C64) {
+            const float g2 = (sm.G[tid] + (tid >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f;
+            sm.G2[tid] = g2;
+            sm.G2r[tid] = g2 - __log2f(sm.rk[tid]);
+        }
+        __syncthreads();
+        const float G31 = sm.G[31];
+        auto Gf = [&](int j) { return sm.G[j] + (j >= 32 ? G31 : 0.f); };
 
-    // ---- A rows into shared memory (warps 0, 1); P rows straight into the record's
-    //      image rows 64-127 (warps 2, 3).  Accumulator row 32 w + lane (warps 0, 1: K K^T,
-    //      2, 3: Q K^T), read eight columns at a time.
-    // erase = 0 (gated linear attention): A = 0, so T = I, which the state kernel's erase =
-    // 0 instance never reads: only the P rows (warps 2, 3) and the vectors are written
-    if (erase || warp >= 2) {
-        const bool arow = warp < 2;
-        const int i = 32 * (warp & 1) + lane;
-        const float Gi2 = sm.G2[i];
-        const float f = arow ? (erase ? sm.beta[i] * sm.rk[i] : 0.f) : sm.rq[i];
-        // rows 0-31 (warps 0, 2) have nothing right of column 31: A there is never read and
-        // the image's P chunks are written as zeros below
-        const int kc_end = (warp & 1) ? 8 : 4;
+        // ---- A rows into shared memory (warps 0, 1); P rows straight into the record's
+        //      image rows 64-127 (warps 2, 3).  Accumulator row 32 w + lane (warps 0, 1: K K^T,
+        //      2, 3: Q K^T), read eight columns at a time.
+        // erase = 0 (gated linear attention): A = 0, so T = I, which the state kernel's erase =
+        // 0 instance never reads: only the P rows (warps 2, 3) and the vectors are written
+        if (erase || warp >= 2) {
+            const bool arow = warp < 2;
+            const int i = 32 * (warp & 1) + lane;
+            const float Gi2 = sm.G2[i];
+            const float f = arow ? (erase ? sm.beta[i] * sm.rk[i] : 0.f) : sm.rq[i];
+            // rows 0-31 (warps 0, 2) have nothing right of column 31: A there is never read and
+            // the image's P chunks are written as zeros below
+            const int kc_end = (warp & 1) ? 8 : 4;
 #pragma unroll 1
-        for (int kc = 0; kc < kc_end; ++kc) {
-            float v[8], p[8];
-            tmem_ld8(tmem + lane_base64(warp) + 8 * kc, v);
-            const float4 g0 = *reinterpret_cast<const float4*>(&sm.G2r[8 * kc]);
-            const float4 g1 = *reinterpret_cast<const float4*>(&sm.G2r[8 * kc + 4]);
-            const float gj[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            tmem_ld_wait();
+            for (int kc = 0; kc < kc_end; ++kc) {
+                float v[8], p[8];
+                tmem_ld8(tmem + lane_base64(warp) + 8 * kc, v);
+                const float4 g0 = *reinterpret_cast<const float4*>(&sm.G2r[8 * kc]);
+                const float4 g1 = *reinterpret_cast<const float4*>(&sm.G2r[8 * kc + 4]);
+                const float gj[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                const int jj = 8 * kc + e;
-                // e^{G_i - G_j} r_k,j = 2^{G2_i - G2r_j}
-                const float2 d = __ffma2_rn(make_float2(gj[e], gj[e + 1]), make_float2(-1.f, -1.f),
-                                            make_float2(Gi2, Gi2));
-                const float2 ex = make_float2(ex2_approx(d.x), ex2_approx(d.y));
-                const float2 pv = __fmul2_rn(__fmul2_rn(make_float2(f, f), ex),
-                                             make_float2(v[e], v[e + 1]));
-                p[e] = (jj < i || (!arow && jj == i)) ? pv.x : 0.f;
-                p[e + 1] = (jj + 1 < i || (!arow && jj + 1 == i)) ? pv.y : 0.f;
-            }
-            if (arow) {
-                *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc]) = make_float4(p[0], p[1], p[2], p[3]);
-                *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc + 4]) = make_float4(p[4], p[5], p[6], p[7]);
-                // A_ba (rows 32-63, columns 0-31) also transposed into the unused top-right
-                // quarter of Am: Am[j][32 + i'] = A[32 + i'][j]
-                if (warp == 1 && kc < 4) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) sm.w.Am[8 * kc + e][32 + lane] = p[e];
+                for (int e = 0; e < 8; e += 2) {
+                    const int jj = 8 * kc + e;
+                    // e^{G_i - G_j} r_k,j = 2^{G2_i - G2r_j}
+                    const float2 d = __ffma2_rn(make_float2(gj[e], gj[e + 1]), make_float2(-1.f, -1.f),
+                                                make_float2(Gi2, Gi2));
+                    const float2 ex = make_float2(ex2_approx(d.x), ex2_approx(d.y));
+                    const float2 pv = __fmul2_rn(__fmul2_rn(make_float2(f, f), ex),
+                                                 make_float2(v[e], v[e + 1]));
+                    p[e] = (jj < i || (!arow && jj == i)) ? pv.x : 0.f;
+                    p[e + 1] = (jj + 1 < i || (!arow && jj + 1 == i)) ? pv.y : 0.f;
                 }
+                if (arow) {
+                    *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc]) = make_float4(p[0], p[1], p[2], p[3]);
+                    *reinterpret_cast<float4*>(&sm.w.Am[i][8 * kc + 4]) =
+                        make_float4(p[4], p[5], p[6], p[7]);
+                    // A_ba (rows 32-63, columns 0-31) also transposed into the unused top-right
+                    // quarter of Am: Am[j][32 + i'] = A[32 + i'][j]
+                    if (warp == 1 && kc < 4) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) sm.w.Am[8 * kc + e][32 + lane] = p[e];
+                    }
+                } else {
+                    store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART,
+                                r64::k_off(C64 + i, kc), p, 1.f);
+                }
+            }
+            if (!arow && kc_end == 4) {
+#pragma unroll
+                for (int kc = 4; kc < 8; ++kc) {
+                    const uint32_t off = r64::k_off(C64 + i, kc);
+                    *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (gi + 1 == grp && warp == 0) tmem_dealloc(tmem, 64);
+        if (erase) {
+            // ---- T = (I + A)^-1.  The four diagonal 16 x 16 blocks by forward substitution, one
+            //      column per lane (warps 0 and 1: lanes 0-15 and 16-31 take one block each);
+            //      warps 2 and 3 zero the blocks above the diagonal.
+            if (warp < 2) {
+                const int o = 32 * warp + (lane & 16), j = lane & 15;
+                float x[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float s0 = i == j ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+                    for (int m = 0; m < (i & ~1); m += 2) {
+                        const float2 av = *reinterpret_cast<const float2*>(&sm.w.Am[o + i][o + m]);
+                        const float2 ss = __ffma2_rn(make_float2(-av.x, -av.y), make_float2(x[m], x[m + 1]),
+                                                     make_float2(s0, s1));
+                        s0 = ss.x;
+                        s1 = ss.y;
+                    }
+                    if (i & 1) s0 -= sm.w.Am[o + i][o + i - 1] * x[i - 1];
+                    x[i] = s0 + s1;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sm.w.Tm[o + i][o + j] = x[i];
             } else {
-                store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(C64 + i, kc), p, 1.f);
-            }
-        }
-        if (!arow && kc_end == 4) {
-#pragma unroll
-            for (int kc = 4; kc < 8; ++kc) {
-                const uint32_t off = r64::k_off(C64 + i, kc);
-                *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 64);
-    if (erase) {
-        // ---- T = (I + A)^-1.  The four diagonal 16 x 16 blocks by forward substitution, one
-        //      column per lane (warps 0 and 1: lanes 0-15 and 16-31 take one block each);
-        //      warps 2 and 3 zero the blocks above the diagonal.
-        if (warp < 2) {
-            const int o = 32 * warp + (lane & 16), j = lane & 15;
-            float x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float s0 = i == j ? 1.f : 0.f, s1 = 0.f;
-#pragma unroll
-                for (int m = 0; m < (i & ~1); m += 2) {
-                    const float2 av = *reinterpret_cast<const float2*>(&sm.w.Am[o + i][o + m]);
-                    const float2 ss = __ffma2_rn(make_float2(-av.x, -av.y), make_float2(x[m], x[m + 1]),
-                                                 make_float2(s0, s1));
-                    s0 = ss.x;
-                    s1 = ss.y;
+                // the zero blocks above the diagonal inside each 32-token block, (0,1) and (2,3),
+                // which the 32-level coupling reads (the upper-right 32 x 32 block of the image is
+                // written as zeros directly)
+                for (int e = tid - 64; e < 2 * 256; e += 64) {
+                    const int blk = e >> 8, w = e & 255, r = w >> 4, cc = w & 15;
+                    sm.w.Tm[32 * blk + r][32 * blk + 16 + cc] = 0.f;
                 }
-                if (i & 1) s0 -= sm.w.Am[o + i][o + i - 1] * x[i - 1];
-                x[i] = s0 + s1;
             }
+            __syncthreads();
+            {
+                // 16-level coupling inside each 32-token block (its triangular solve):
+                // Z = A[b+16.., b..] T[b.., b..], thread -> (block bi, row i, 4 columns)
+                const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
+                float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sm.w.Tm[o + i][o + j] = x[i];
-        } else {
-            // the zero blocks above the diagonal inside each 32-token block, (0,1) and (2,3),
-            // which the 32-level coupling reads (the upper-right 32 x 32 block of the image is
-            // written as zeros directly)
-            for (int e = tid - 64; e < 2 * 256; e += 64) {
-                const int blk = e >> 8, w = e & 255, r = w >> 4, cc = w & 15;
-                sm.w.Tm[32 * blk + r][32 * blk + 16 + cc] = 0.f;
+                for (int m = 0; m < 16; ++m) {
+                    const float a_ = sm.w.Am[o + 16 + i][o + m];
+                    const float4 t4 = *reinterpret_cast<const float4*>(&sm.w.Tm[o + m][o + jc]);
+                    const float2 a2 = make_float2(a_, a_);
+                    const float2 z01 = __ffma2_rn(a2, make_float2(t4.x, t4.y), make_float2(z[0], z[1]));
+                    const float2 z23 = __ffma2_rn(a2, make_float2(t4.z, t4.w), make_float2(z[2], z[3]));
+                    z[0] = z01.x; z[1] = z01.y; z[2] = z23.x; z[3] = z23.y;
+                }
+                *reinterpret_cast<float4*>(&sm.w.Am[o + i][o + jc]) = make_float4(z[0], z[1], z[2], z[3]);
             }
-        }
-        __syncthreads();
-        {
-            // 16-level coupling inside each 32-token block (its triangular solve):
-            // Z = A[b+16.., b..] T[b.., b..], thread -> (block bi, row i, 4 columns)
-            const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
-            float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float a_ = sm.w.Am[o + 16 + i][o + m];
-                const float4 t4 = *reinterpret_cast<const float4*>(&sm.w.Tm[o + m][o + jc]);
-                const float2 z01 = __ffma2_rn(make_float2(a_, a_), make_float2(t4.x, t4.y), make_float2(z[0], z[1]));
-                const float2 z23 = __ffma2_rn(make_float2(a_, a_), make_float2(t4.z, t4.w), make_float2(z[2], z[3]));
-                z[0] = z01.x; z[1] = z01.y; z[2] = z23.x; z[3] = z23.y;
-            }
-            *reinterpret_cast<float4*>(&sm.w.Am[o + i][o + jc]) = make_float4(z[0], z[1], z[2], z[3]);
-        }
-        __syncthreads();
-        {
-            // T[b+16.., b..] = -T[b+16.., b+16..] Z.  That block is lower triangular: row i needs
-            // m <= i only; a warp's rows end at 7 or 15, and the zero upper triangle it still
-            // reads below that is stored.
-            const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
-            const int mend = (warp & 1) ? 16 : 8;
-            float t[4] = {0.f, 0.f, 0.f, 0.f};
+            __syncthreads();
+            {
+                // T[b+16.., b..] = -T[b+16.., b+16..] Z.  That block is lower triangular: row i needs
+                // m <= i only; a warp's rows end at 7 or 15, and the zero upper triangle it still
+                // reads below that is stored.
+                const int bi = tid >> 6, i = (tid >> 2) & 15, jc = 4 * (tid & 3), o = 32 * bi;
+                const int mend = (warp & 1) ? 16 : 8;
+                float t[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-            for (int m = 0; m < mend; ++m) {
-                const float tv = sm.w.Tm[o + 16 + i][o + 16 + m];
-                const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Am[o + m][o + jc]);
-                const float2 t01 = __ffma2_rn(make_float2(tv, tv), make_float2(z4.x, z4.y), make_float2(t[0], t[1]));
-                const float2 t23 = __ffma2_rn(make_float2(tv, tv), make_float2(z4.z, z4.w), make_float2(t[2], t[3]));
-                t[0] = t01.x; t[1] = t01.y; t[2] = t23.x; t[3] = t23.y;
+                for (int m = 0; m < mend; ++m) {
+                    const float tv = sm.w.Tm[o + 16 + i][o + 16 + m];
+                    const float4 z4 = *reinterpret_cast<const float4*>(&sm.w.Am[o + m][o + jc]);
+                    const float2 tv2 = make_float2(tv, tv);
+                    const float2 t01 = __ffma2_rn(tv2, make_float2(z4.x, z4.y), make_float2(t[0], t[1]));
+                    const float2 t23 = __ffma2_rn(tv2, make_float2(z4.z, z4.w), make_float2(t[2], t[3]));
+                    t[0] = t01.x; t[1] = t01.y; t[2] = t23.x; t[3] = t23.y;
+                }
+                *reinterpret_cast<float4*>(&sm.w.Tm[o + 16 + i][o + jc]) =
+                    make_float4(-t[0], -t[1], -t[2], -t[3]);
             }
-            *reinterpret_cast<float4*>(&sm.w.Tm[o + 16 + i][o + jc]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
-        }
-        __syncthreads();
-        {
-            // 32-level coupling: Z = A_ba T_a (rows 32-63, columns 0-31), warp w -> columns
-            // 8 w .. 8 w + 7, lane -> row.  T_a is lower triangular: column j needs m >= j, so
-            // the warp starts at m = 8 w (the zeros it reads above the diagonal are stored);
-            // A_ba comes from its transposed copy (consecutive lanes, consecutive words).
-            const int i = lane, j0 = 8 * warp;
-            float z[8];
+            __syncthreads();
+            {
+                // 32-level coupling: Z = A_ba T_a (rows 32-63, columns 0-31), warp w -> columns
+                // 8 w .. 8 w + 7, lane -> row.  T_a is lower triangular: column j needs m >= j, so
+                // the warp starts at m = 8 w (the zeros it reads above the diagonal are stored);
+                // A_ba comes from its transposed copy (consecutive lanes, consecutive words).
+                const int i = lane, j0 = 8 * warp;
+                float z[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) z[q] = 0.f;
+                for (int q = 0; q < 8; ++q) z[q] = 0.f;
 #pragma unroll 4
-            for (int m = j0; m < 32; ++m) {
-                const float a_ = sm.w.Am[m][32 + i];
-                const float4 t0v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0]);
-                const float4 t1v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0 + 4]);
-                const float2 a2 = make_float2(a_, a_);
-                const float2 za = __ffma2_rn(a2, make_float2(t0v.x, t0v.y), make_float2(z[0], z[1]));
-                const float2 zb = __ffma2_rn(a2, make_float2(t0v.z, t0v.w), make_float2(z[2], z[3]));
-                const float2 zc = __ffma2_rn(a2, make_float2(t1v.x, t1v.y), make_float2(z[4], z[5]));
-                const float2 zd = __ffma2_rn(a2, make_float2(t1v.z, t1v.w), make_float2(z[6], z[7]));
-                z[0] = za.x; z[1] = za.y; z[2] = zb.x; z[3] = zb.y;
-                z[4] = zc.x; z[5] = zc.y; z[6] = zd.x; z[7] = zd.y;
+                for (int m = j0; m < 32; ++m) {
+                    const float a_ = sm.w.Am[m][32 + i];
+                    const float4 t0v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0]);
+                    const float4 t1v = *reinterpret_cast<const float4*>(&sm.w.Tm[m][j0 + 4]);
+                    const float2 a2 = make_float2(a_, a_);
+                    const float2 za = __ffma2_rn(a2, make_float2(t0v.x, t0v.y), make_float2(z[0], z[1]));
+                    const float2 zb = __ffma2_rn(a2, make_float2(t0v.z, t0v.w), make_float2(z[2], z[3]));
+                    const float2 zc = __ffma2_rn(a2, make_float2(t1v.x, t1v.y), make_float2(z[4], z[5]));
+                    const float2 zd = __ffma2_rn(a2, make_float2(t1v.z, t1v.w), make_float2(z[6], z[7]));
+                    z[0] = za.x; z[1] = za.y; z[2] = zb.x; z[3] = zb.y;
+                    z[4] = zc.x; z[5] = zc.y; z[6] = zd.x; z[7] = zd.y;
+                }
+                *reinterpret_cast<float4*>(&sm.w.Am[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
+                *reinterpret_cast<float4*>(&sm.w.Am[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
             }
-            *reinterpret_cast<float4*>(&sm.w.Am[i][j0]) = make_float4(z[0], z[1], z[2], z[3]);
-            *reinterpret_cast<float4*>(&sm.w.Am[i][j0 + 4]) = make_float4(z[4], z[5], z[6], z[7]);
-        }
-        __syncthreads();
-        {
-            // T_ba = -T_b Z.  T_b is lower triangular: row i needs m <= i only; warp w holds rows
-            // 8 w .. 8 w + 7 (the zero upper triangle it reads below 8 w + 8 is stored).
-            const int i = tid >> 2, j0 = 8 * (tid & 3);
-            float t[8];
+            __syncthreads();
+            {
+                // T_ba = -T_b Z.  T_b is lower triangular: row i needs m <= i only; warp w holds rows
+                // 8 w .. 8 w + 7 (the zero upper triangle it reads below 8 w + 8 is stored).
+                const int i = tid >> 2, j0 = 8 * (tid & 3);
+                float t[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) t[q] = 0.f;
+                for (int q = 0; q < 8; ++q) t[q] = 0.f;
 #pragma unroll 4
-            for (int m = 0; m < 8 * warp + 8; ++m) {
-                const float tv = sm.w.Tm[32 + i][32 + m];
-                const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0]);
-                const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0 + 4]);
-                const float2 t2 = make_float2(tv, tv);
-                const float2 ta = __ffma2_rn(t2, make_float2(z0.x, z0.y), make_float2(t[0], t[1]));
-                const float2 tb = __ffma2_rn(t2, make_float2(z0.z, z0.w), make_float2(t[2], t[3]));
-                const float2 tc_ = __ffma2_rn(t2, make_float2(z1.x, z1.y), make_float2(t[4], t[5]));
-                const float2 td = __ffma2_rn(t2, make_float2(z1.z, z1.w), make_float2(t[6], t[7]));
-                t[0] = ta.x; t[1] = ta.y; t[2] = tb.x; t[3] = tb.y;
-                t[4] = tc_.x; t[5] = tc_.y; t[6] = td.x; t[7] = td.y;
+                for (int m = 0; m < 8 * warp + 8; ++m) {
+                    const float tv = sm.w.Tm[32 + i][32 + m];
+                    const float4 z0 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0]);
+                    const float4 z1 = *reinterpret_cast<const float4*>(&sm.w.Am[m][j0 + 4]);
+                    const float2 t2 = make_float2(tv, tv);
+                    const float2 ta = __ffma2_rn(t2, make_float2(z0.x, z0.y), make_float2(t[0], t[1]));
+                    const float2 tb = __ffma2_rn(t2, make_float2(z0.z, z0.w), make_float2(t[2], t[3]));
+                    const float2 tc_ = __ffma2_rn(t2, make_float2(z1.x, z1.y), make_float2(t[4], t[5]));
+                    const float2 td = __ffma2_rn(t2, make_float2(z1.z, z1.w), make_float2(t[6], t[7]));
+                    t[0] = ta.x; t[1] = ta.y; t[2] = tb.x; t[3] = tb.y;
+                    t[4] = tc_.x; t[5] = tc_.y; t[6] = td.x; t[7] = td.y;
+                }
+                *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+                *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0 + 4]) =
+                    make_float4(-t[4], -t[5], -t[6], -t[7]);
             }
-            *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0]) = make_float4(-t[0], -t[1], -t[2], -t[3]);
-            *reinterpret_cast<float4*>(&sm.w.Tm[32 + i][j0 + 4]) = make_float4(-t[4], -t[5], -t[6], -t[7]);
-        }
-        __syncthreads();
-        // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread); rows 0-31 x
-        //      columns 32-63 are zero.  Eight consecutive lanes take the eight rows of one
-        //      8-row group at one chunk: one 128-byte line of the image.
+            __syncthreads();
+            // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread); rows 0-31 x
+            //      columns 32-63 are zero.  Eight consecutive lanes take the eight rows of one
+            //      8-row group at one chunk: one 128-byte line of the image.
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int task = tid + PREP64_THREADS * e;
-            const int row = 8 * (task >> 6) + (task & 7), kc = (task >> 3) & 7;
-            if (row < 32 && kc >= 4) {
-                const uint32_t off = r64::k_off(row, kc);
-                *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
-            } else {
-                store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(row, kc),
-                            &sm.w.Tm[row][8 * kc], -1.f);
+            for (int e = 0; e < 4; ++e) {
+                const int task = tid + PREP64_THREADS * e;
+                const int row = 8 * (task >> 6) + (task & 7), kc = (task >> 3) & 7;
+                if (row < 32 && kc >= 4) {
+                    const uint32_t off = r64::k_off(row, kc);
+                    *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
+                } else {
+                    store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(row, kc),
+                                &sm.w.Tm[row][8 * kc], -1.f);
+                }
             }
+        }  // erase
+        // the next head's gate inputs (warps 2, 3) while warps 0, 1 write the vectors: a
+        // block barrier waits for a thread's loads, and the next one is at the loop's top
+        if (gi + 1 < grp) load_gates(h + 1);
+        // ---- vectors
+        if (tid < C64) {
+            const int i = tid;
+            float* vec = reinterpret_cast<float*>(rc + r64::OFF_VEC);
+            const float Gi = Gf(i), GC = Gf(C64 - 1), eG = __expf(Gi);
+            vec[r64::VEC_E + i] = eG * sm.rq[i];
+            vec[r64::VEC_D + i] = __expf(GC - Gi) * sm.rk[i];
+            vec[r64::VEC_BETA + i] = sm.beta[i];
+            vec[r64::VEC_W + i] = erase ? sm.beta[i] * eG * sm.rk[i] : 0.f;
+            if (i == 0) vec[r64::VEC_GAMMA] = __expf(GC);
         }
-    }  // erase
-    // ---- vectors
-    if (tid < C64) {
-        const int i = tid;
-        float* vec = reinterpret_cast<float*>(rc + r64::OFF_VEC);
-        const float Gi = Gf(i), GC = Gf(C64 - 1), eG = __expf(Gi);
-        vec[r64::VEC_E + i] = eG * sm.rq[i];
-        vec[r64::VEC_D + i] = __expf(GC - Gi) * sm.rk[i];
-        vec[r64::VEC_BETA + i] = sm.beta[i];
-        vec[r64::VEC_W + i] = erase ? sm.beta[i] * eG * sm.rk[i] : 0.f;
-        if (i == 0) vec[r64::VEC_GAMMA] = __expf(GC);
-    }
+    }  // value heads of the key head
 }
 
 // ================================================================= state-passing kernel
@@ -1230,7 +1263,7 @@ cudaError_t prepare64(const FwdParams& p, Maps64& m) {
 
 cudaError_t launch_intra64(const FwdParams& p, const Maps64& m, void* ws, cudaStream_t stream) {
     const long long nrec = r64::max_records(p.cu_seqlens != nullptr, p.nseq, p.T);
-    intra64_kernel<<<(unsigned)(nrec * p.Hv), PREP64_THREADS, sizeof(Prep64Smem), stream>>>(
+    intra64_kernel<<<(unsigned)(nrec * p.Hk), PREP64_THREADS, sizeof(Prep64Smem), stream>>>(
         m.q, m.k, (const __nv_bfloat16*)p.a, (const __nv_bfloat16*)p.b, p.A_log, p.dt_bias,
         p.cu_seqlens, p.T, p.nseq, p.Hk, p.Hv, p.erase, (uint8_t*)ws);
     return cudaGetLastError();
