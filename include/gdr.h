@@ -149,7 +149,8 @@ GDR_API int gdr_prefill_chunked_noalloc(const void* q, const void* k, const void
 /*
  * The maps of B segments (dense [B, T] or packed with cu_seqlens, exactly as the
  * sequences of gdr_prefill_chunked): phi [B, Hv, dk, dk] and nmap [B, Hv, dk, dv], fp32.
- * No output is written.  Runs the tensor-core prefill twice; T >= 1.
+ * No output is written.  One intra-block pass, then one state pass that runs both maps
+ * over its records; T >= 1.
  */
 GDR_API int gdr_prefill_segment_maps(const void* q, const void* k, const void* v,
                                      const void* a, const void* b, const float* A_log,
@@ -175,10 +176,11 @@ GDR_API int gdr_segment_combine(const float* phi, const float* nmap, const float
  * [1, Hv, dk, dv], nullable as in gdr_prefill_chunked) cut into at most nseg
  * chunk-aligned segments that run side by side on this device: segment maps, their
  * composition, then the prefill of every segment from its start state.  Same results as
- * gdr_prefill_chunked up to rounding; it does about three times the work, in
- * T / nseg-long chains instead of one T-long chain, which pays when the sequences x
- * heads of a call leave most of the GPU idle (few heads, long context).  Workspace:
- * 3 nseg Hv 64 KB from the pool described at the top of this file, plus the prefill's.
+ * gdr_prefill_chunked up to rounding; it does about three state passes of work (the two
+ * maps, then the segments' prefill on the same intra-block records), in T / nseg-long
+ * chains instead of one T-long chain, which pays when the sequences x heads of a call
+ * leave most of the GPU idle (few heads, long context).  Workspace: 3 nseg Hv 64 KB from
+ * the pool described at the top of this file, plus the prefill's records.
  */
 GDR_API int gdr_prefill_chunked_cp(const void* q, const void* k, const void* v, const void* a,
                                    const void* b, const float* A_log, const float* dt_bias,
