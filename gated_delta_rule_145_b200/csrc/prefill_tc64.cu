@@ -571,6 +571,9 @@ constexpr int O_PITCH = 52;             // floats: 208 B rows, 16-byte aligned
 //   19             issues [K; Q] [S hi | lo] (meets the S group on BAR_S) and the loads:
 //                  TMA tiles [K; Q] and V, the record image [-T; P] and its vectors,
 //                  two-deep ring
+// The erase = 0 instance (kGla): no Delta product; the BD group writes D Delta and Delta
+// from V (no K S), warp 18 issues G3 and P Delta on one barrier with it, and warp 8 issues
+// the loads after the first two blocks (a block ahead of the state, as the slot frees).
 struct alignas(1024) Sp64Smem {
     uint8_t kq[2][32768];   // block s: per dk half (16 KB) K rows 0-63 | Q rows 64-127
     uint8_t rec[2][32768];  // block s: [-T; P] hi (16 KB), lo (16 KB)

@@ -96,6 +96,21 @@ def test_prefill_dense_block_multiples(T):
     _check_prefill(inp, "chunked")
 
 
+@pytest.mark.parametrize("erase", [True, False])
+def test_prefill_one_key_head_for_eight_value_heads(erase):
+    """The intra-block kernel computes a key head's tiles, Gram and norms once and then
+    each of its value heads in turn: Hk=1 shared by Hv=8, a ragged dense batch."""
+    inp = synth.make_inputs(2, 150, 1, 8, 128, 128, "bf16", seed=17, s0_std=0.05)
+    d = to_device(inp)
+    out, fin = gdr.prefill(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                           d["init_state"], erase=erase)
+    torch.cuda.synchronize()
+    assert gdr.gdr_device_status() == gdr.GDR_OK
+    ro, rS = oracle_forward(inp, erase=erase)
+    assert_parity(_np(out), ro, TAU["bf16"], f"Hk=1 Hv=8 o (erase={erase})")
+    assert_parity(_np(fin), rS, TAU["bf16"], f"Hk=1 Hv=8 S (erase={erase})")
+
+
 def test_zero_length_returns_initial_state():
     inp = synth.make_inputs(3, 0, 2, 2, 128, 128, "bf16", seed=10, s0_std=0.1)
     for form in ("chunked", "recurrent"):
