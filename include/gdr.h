@@ -43,6 +43,11 @@
  *     stream once the call's kernels are enqueued).  Freed memory stays cached in the pool
  *     for later calls until gdr_release_workspace().  Calls on different streams get
  *     different workspace memory.  No other call allocates device memory.
+ *   - CUDA graphs: the device-buffer calls enqueue only kernels (and, for the prefill, the
+ *     pool allocation and free) on `stream`, so they may be captured in a graph and
+ *     replayed; the replay gives the direct call's results bit for bit (tested for
+ *     gdr_decode_step and gdr_prefill_chunked).  A decode loop replayed from a graph pays
+ *     no host work per step.
  */
 #ifndef GDR_H_
 #define GDR_H_
