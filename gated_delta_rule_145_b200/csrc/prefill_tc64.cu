@@ -279,7 +279,9 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncwarp();
     }
     // ---- inverse norms of the K rows (0-63) and Q rows (64-127): a thread pair per row
-    //      (the swizzle only permutes 16-byte pieces inside a row, which a sum ignores)
+    //      (the swizzle only permutes 16-byte pieces inside a row, which a sum ignores);
+    //      with them the first value head's exponents (later heads: at the loop's top)
+    if (tid < C64) sm.G2[tid] = (sm.G[tid] + (tid >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f;
     if (ok) {
 #pragma unroll 1
         for (int e = 0; e < 2; ++e) {
@@ -288,7 +290,10 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ss += __shfl_xor_sync(0xffffffffu, ss, 1);
             if (hf == 0) {
                 if (e == 0) {
-                    sm.rk[row] = rsqrtf(ss + kNormEps);
+                    const float r = rsqrtf(ss + kNormEps);
+                    sm.rk[row] = r;
+                    sm.G2r[row] = (sm.G[row] + (row >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f -
+                                  __log2f(r);
                 } else {
                     sm.rq[row - 64] = rsqrtf(ss + kNormEps) * rsqrtf((float)DK);
                 }
@@ -309,16 +314,16 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (gi > 0) {
             __syncthreads();  // the previous head's last phase has read G and beta
             gates();
+            __syncthreads();
+            // the block's G times log2(e), and with -log2(r_k): a column's decay and key
+            // scale in one exponent
+            if (tid < C64) {
+                const float g2 = (sm.G[tid] + (tid >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f;
+                sm.G2[tid] = g2;
+                sm.G2r[tid] = g2 - __log2f(sm.rk[tid]);
+            }
+            __syncthreads();
         }
-        __syncthreads();
-        // the block's G times log2(e), and with -log2(r_k): a column's decay and key scale in
-        // one exponent
-        if (tid < C64) {
-            const float g2 = (sm.G[tid] + (tid >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f;
-            sm.G2[tid] = g2;
-            sm.G2r[tid] = g2 - __log2f(sm.rk[tid]);
-        }
-        __syncthreads();
         const float G31 = sm.G[31];
         auto Gf = [&](int j) { return sm.G[j] + (j >= 32 ? G31 : 0.f); };
 
