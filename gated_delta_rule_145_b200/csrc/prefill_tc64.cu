@@ -64,10 +64,16 @@ constexpr uint32_t VEC_BYTES = 1040;        // 257 floats, padded to 16 bytes
 constexpr uint32_t BYTES = 2 * PART + VEC_BYTES;
 
 // Byte offset of row m, K-chunk kc (8 elements) in a K-major no-swizzle image of 8 chunks
-// per row: core matrices of 8 rows x 16 bytes, the 8 chunks of an 8-row group contiguous.
+// per row: core matrices of 8 rows x 16 bytes; chunks 0-3 of all 16 row groups first, then
+// chunks 4-7 (an MMA's K = 16 takes two chunks of one half: chunk stride 128 bytes, row
+// group stride 512).  Rows 0-31 of -T and of P are zero in chunks 4-7, so each part holds
+// two 2 KB zero ranges that are neither written nor loaded.
 __host__ __device__ constexpr uint32_t k_off(int m, int kc) {
-    return (uint32_t)((m / 8) * 1024 + kc * 128 + (m % 8) * 16);
+    return (uint32_t)((kc / 4) * 8192 + (m / 8) * 512 + (kc % 4) * 128 + (m % 8) * 16);
 }
+constexpr uint32_t ZERO_A = 8192;   // rows 0-31 (-T), chunks 4-7: [ZERO_A, ZERO_A + 2048)
+constexpr uint32_t ZERO_P = 12288;  // rows 64-95 (P rows 0-31), chunks 4-7
+constexpr uint32_t ZERO_BYTES = 2048;
 
 __host__ __device__ constexpr long long max_records(bool varlen, int nseq, int T) {
     return varlen ? ((long long)T + 63LL * nseq) / C64 + 1 : (long long)nseq * ((T + C64 - 1) / C64);
@@ -375,12 +381,15 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 r64::k_off(C64 + i, kc), p, 1.f);
                 }
             }
-            if (!arow && kc_end == 4) {
+            // erase = 0: P's rows 0-31 are zero in chunks 4-7 as well, but that instance loads
+            // the P rows in one piece, zero range included
+            if (!erase && !arow && kc_end == 4) {
 #pragma unroll
                 for (int kc = 4; kc < 8; ++kc) {
                     const uint32_t off = r64::k_off(C64 + i, kc);
                     *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) =
+                        make_uint4(0, 0, 0, 0);
                 }
             }
         }
@@ -509,20 +518,16 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             __syncthreads();
             // ---- image rows 0-63: -T (64 rows x 8 chunks, four chunks per thread); rows 0-31 x
-            //      columns 32-63 are zero.  Eight consecutive lanes take the eight rows of one
-            //      8-row group at one chunk: one 128-byte line of the image.
+            //      columns 32-63 are zero and not written (the state kernel keeps zeros
+            //      there).  Eight consecutive lanes take the eight rows of one 8-row group at
+            //      one chunk: one 128-byte line of the image.
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int task = tid + PREP64_THREADS * e;
                 const int row = 8 * (task >> 6) + (task & 7), kc = (task >> 3) & 7;
-                if (row < 32 && kc >= 4) {
-                    const uint32_t off = r64::k_off(row, kc);
-                    *reinterpret_cast<uint4*>(rc + r64::OFF_A + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(rc + r64::OFF_A + r64::PART + off) = make_uint4(0, 0, 0, 0);
-                } else {
+                if (row >= 32 || kc < 4)
                     store_chunk(rc + r64::OFF_A, rc + r64::OFF_A + r64::PART, r64::k_off(row, kc),
                                 &sm.w.Tm[row][8 * kc], -1.f);
-                }
             }
         }  // erase
         // the next head's gate inputs (warps 2, 3) while warps 0, 1 write the vectors: a
@@ -723,8 +728,10 @@ __device__ void issue_loads(Sp64Smem& sm, const Sp64Ctx& x, int s, const CUtenso
                             const CUtensorMap* tm_k, const CUtensorMap* tm_v) {
     const int r = s & 1;
     uint64_t* bar = &sm.full[r];
-    // erase = 0: the record's -T rows (0-63) are neither written nor read
-    const uint32_t part = x.gla ? r64::PART / 2 : r64::PART;
+    // the image parts without their zero ranges; erase = 0: P's rows only, [4096, 16384)
+    // with its zero range (which that instance's intra-block kernel writes) in one piece; the
+    // -T rows are neither written nor read
+    const uint32_t part = x.gla ? r64::PART - 4096u : r64::PART - 2 * r64::ZERO_BYTES;
     mbar_arrive_expect_tx(bar, (x.v_zero ? 8u : 10u) * 4096u + 2u * part + r64::VEC_BYTES);
     const int y = (int)(x.t0 + (long long)s * C64);
 #pragma unroll 1
@@ -741,9 +748,20 @@ __device__ void issue_loads(Sp64Smem& sm, const Sp64Ctx& x, int s, const CUtenso
         tma_load_2d(sm.vt[r] + 4096, tm_v, x.h * DV + x.col0, y + 32, bar);
     }
     const uint8_t* rc = x.record(s);
-    const uint32_t skip = r64::PART - part;  // rows 0-63 are the first half of a part
-    bulk_load(sm.rec[r] + skip, rc + r64::OFF_A + skip, part, bar);
-    bulk_load(sm.rec[r] + r64::PART + skip, rc + r64::OFF_A + r64::PART + skip, part, bar);
+#pragma unroll 1
+    for (uint32_t h = 0; h < 2 * r64::PART; h += r64::PART) {
+        const uint8_t* src = rc + r64::OFF_A + h;
+        uint8_t* dst = sm.rec[r] + h;
+        if (x.gla) {
+            bulk_load(dst + 4096, src + 4096, r64::PART - 4096, bar);
+            continue;
+        }
+        bulk_load(dst, src, r64::ZERO_A, bar);
+        bulk_load(dst + r64::ZERO_A + r64::ZERO_BYTES, src + r64::ZERO_A + r64::ZERO_BYTES,
+                  r64::ZERO_P - r64::ZERO_A - r64::ZERO_BYTES, bar);
+        bulk_load(dst + r64::ZERO_P + r64::ZERO_BYTES, src + r64::ZERO_P + r64::ZERO_BYTES,
+                  r64::PART - r64::ZERO_P - r64::ZERO_BYTES, bar);
+    }
     bulk_load(sm.vec[r], rc + r64::OFF_VEC, r64::VEC_BYTES, bar);
 }
 
@@ -812,7 +830,7 @@ __device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
     const uint32_t id96 = idesc_bf16(128, 2 * NT, 0, 1);
     const uint32_t id48 = idesc_bf16(128, NT, 0, 1);
     const uint32_t id_g3 = idesc_bf16(128, 2 * NT, 1, 1);
-    const uint64_t d_rec = sdesc(smem_u32(sm.rec[0]), 128, 1024, kSwNone);   // [-T; P] K-major
+    const uint64_t d_rec = sdesc(smem_u32(sm.rec[0]), 128, 512, kSwNone);    // [-T; P] K-major
     const uint64_t d_kt = sdesc(smem_u32(sm.kq[0]), 16384, 1024, kSw128);    // K^T MN-major
     const uint64_t d_b = sdesc(smem_u32(sm.b_op), 128, 1024, kSwNone);
     const uint64_t d_d = sdesc(smem_u32(sm.d_op), 128, 1024, kSwNone);
@@ -823,11 +841,12 @@ __device__ void d_issue_role(Sp64Smem& sm, const Sp64Ctx& x, int lane) {
     auto tp_product = [&](int r, uint32_t dcol, uint64_t dx) {
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(x.tmem + dcol, dadd64(d_rec, r * 32768 + ks * 256), dadd64(dx, ks * 256), id96,
-                     ks > 0);
+            mma_bf16(x.tmem + dcol, dadd64(d_rec, r * 32768 + (ks >> 1) * 8192 + (ks & 1) * 256),
+                     dadd64(dx, ks * 256), id96, ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(x.tmem + dcol, dadd64(d_rec, r * 32768 + r64::PART + ks * 256),
+            mma_bf16(x.tmem + dcol,
+                     dadd64(d_rec, r * 32768 + r64::PART + (ks >> 1) * 8192 + (ks & 1) * 256),
                      dadd64(dx, ks * 256), id48, 1);
     };
     bool live = true;
@@ -1199,6 +1218,13 @@ state64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tma_prefetch_map(&tm_k);
         tma_prefetch_map(&tm_v);
     }
+    // the zero ranges of the record images, which the loads skip: both slots, hi and lo
+    for (int i = tid; i < 2 * 2 * 2 * (int)(r64::ZERO_BYTES / 16); i += SP_THREADS) {
+        const int slot = i >> 9, part = (i >> 8) & 1, zr = (i >> 7) & 1, c16 = i & 127;
+        *reinterpret_cast<uint4*>(sm.rec[slot] + part * r64::PART + (zr ? r64::ZERO_P : r64::ZERO_A) +
+                                  16 * c16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_async_smem();
     if (warp == 0) tmem_alloc(&sm.tmem_base, TMEM_COLS);
     tc_fence_before();
     __syncthreads();
