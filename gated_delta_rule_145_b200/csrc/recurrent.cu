@@ -72,6 +72,10 @@ recurrent_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
                  const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv, int erase) {
     using Sh = RecShape<DK, DV, Tin>;
     constexpr int COLS = Sh::COLS, CG = Sh::CG, RG = Sh::RG, RPT = Sh::RPT, EPL = Sh::EPL;
+    // launched with programmatic stream serialization: let the next launch be scheduled,
+    // and wait for everything before this one in the stream before reading anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int NSLICE = DV / COLS;
     const int slice = blockIdx.x % NSLICE;
     const int h = (blockIdx.x / NSLICE) % Hv;
@@ -189,12 +193,19 @@ recurrent_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
 template <int D, typename Tin>
 cudaError_t launch_typed(const FwdParams& p, cudaStream_t stream) {
     using Sh = RecShape<D, D, Tin>;
-    const dim3 grid((unsigned)(p.nseq * p.Hv * (D / Sh::COLS)));
-    recurrent_kernel<D, D, Tin><<<grid, Sh::NT, 0, stream>>>(
-        (const Tin*)p.q, (const Tin*)p.k, (const Tin*)p.v, (const Tin*)p.a, (const Tin*)p.b,
-        p.A_log, p.dt_bias, p.init_state, p.out, p.final_state, p.cu_seqlens, p.T, p.Hk, p.Hv,
-        p.erase);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.nseq * p.Hv * (D / Sh::COLS)));
+    cfg.blockDim = dim3(Sh::NT);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, recurrent_kernel<D, D, Tin>, (const Tin*)p.q, (const Tin*)p.k,
+                              (const Tin*)p.v, (const Tin*)p.a, (const Tin*)p.b, p.A_log,
+                              p.dt_bias, p.init_state, p.out, p.final_state, p.cu_seqlens, p.T,
+                              p.Hk, p.Hv, p.erase);
 }
 
 template <typename Tin>
