@@ -72,8 +72,9 @@ recurrent_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
                  const int32_t* __restrict__ cu_seqlens, int T, int Hk, int Hv, int erase) {
     using Sh = RecShape<DK, DV, Tin>;
     constexpr int COLS = Sh::COLS, CG = Sh::CG, RG = Sh::RG, RPT = Sh::RPT, EPL = Sh::EPL;
-    // launched with programmatic stream serialization: let the next launch be scheduled,
-    // and wait for everything before this one in the stream before reading anything
+    // launched with programmatic stream serialization (grids of several waves): let the
+    // next launch be scheduled, and wait for everything before this one in the stream before
+    // reading anything (both are no-ops for a launch without it)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int NSLICE = DV / COLS;
@@ -190,18 +191,32 @@ recurrent_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     }
 }
 
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
 template <int D, typename Tin>
 cudaError_t launch_typed(const FwdParams& p, cudaStream_t stream) {
     using Sh = RecShape<D, D, Tin>;
+    const long long grid = (long long)p.nseq * p.Hv * (D / Sh::COLS);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.nseq * p.Hv * (D / Sh::COLS)));
+    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(Sh::NT);
     cfg.stream = stream;
+    // programmatic serialization pays where a launch runs several waves (its successor's
+    // CTAs fill the last wave's idle slots); a grid of one wave or less only waits longer
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = grid >= 8LL * sm_count() ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, recurrent_kernel<D, D, Tin>, (const Tin*)p.q, (const Tin*)p.k,
                               (const Tin*)p.v, (const Tin*)p.a, (const Tin*)p.b, p.A_log,
                               p.dt_bias, p.init_state, p.out, p.final_state, p.cu_seqlens, p.T,
