@@ -13,8 +13,10 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 
-def test_decode_steps_replayed_from_a_graph_match_direct_calls():
-    B, H, D, n = 2, 4, 128, 8
+# B=64, H=48: a grid of several waves, launched with programmatic stream serialization
+@pytest.mark.parametrize("B,H,n", [(2, 4, 8), (64, 48, 4)])
+def test_decode_steps_replayed_from_a_graph_match_direct_calls(B, H, n):
+    D = 128
     inp = synth.make_inputs(B, n, H, H, D, D, "bf16", seed=71, s0_std=0.05)
     dev = torch.device("cuda", 0)
 
