@@ -1,5 +1,6 @@
 // mixer_io.cu -- the steps on either side of the gated delta rule in its mixer:
-//   short_conv_silu_kernel  before it: a short causal depthwise convolution over time
+//   short_conv_silu_tiled_kernel / short_conv_silu_kernel
+//                           before it: a short causal depthwise convolution over time
 //                           (four taps, kept as a ring buffer of the last three inputs
 //                           per channel) followed by SiLU, on the input projections;
 //   gated_rmsnorm_kernel    after it: RMS normalisation of each head's output over the

@@ -16,9 +16,11 @@
 //     o     = gamma p + (q . k) delta        ( = q^T S_new )
 //     S_new = gamma S_old + k delta^T
 // so S is touched once per step.  Without the erase term (erase = 0: gated linear
-// attention, the erase=False case of tessera PR #77 summary, "What landed") delta = beta v.  Every warp normalises q and k itself (warp reductions,
-// no block barrier); the column sums over row groups cross warps through a double-
-// buffered shared array, one block barrier per token.
+// attention, the erase=False case of tessera PR #77 summary, "What landed") delta = beta v.
+// Every warp normalises q and k itself (warp reductions, no block barrier); the column
+// sums over row groups cross warps through a double-buffered shared array, one block
+// barrier per token.  Grids of several waves (a decode batch) launch with programmatic
+// stream serialization, so a step's CTAs fill the previous step's last wave.
 #include "gdr_common.cuh"
 #include "gdr_internal.h"
 
