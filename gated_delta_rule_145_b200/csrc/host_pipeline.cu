@@ -20,6 +20,8 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "gdr_internal.h"
 
@@ -95,7 +97,19 @@ cudaError_t launch_prefill_host(const FwdParams& hp, int seg, cudaStream_t strea
     const size_t rq = (size_t)Hk * dk * eb, rv = (size_t)Hv * dv * eb, rg = (size_t)Hv * eb;
     const size_t ro = (size_t)Hv * dv * sizeof(float);
     const size_t st = (size_t)B * Hv * dk * dv * sizeof(float);
-    const int nseg = (T + seg - 1) / seg;
+    // Chunk-aligned segments of `seg` tokens; the last one is cut in two, twice (first
+    // parts a multiple of 32 tokens and at least 128), so that the final copy-out, which
+    // nothing overlaps, is a quarter of a segment.
+    std::vector<std::pair<int, int>> segs;  // (first token, tokens)
+    for (int t0 = 0; t0 < T; t0 += seg) segs.emplace_back(t0, T - t0 < seg ? T - t0 : seg);
+    for (int cut = 0; cut < 2 && segs.size() >= 2; ++cut) {
+        const int t0 = segs.back().first, n = segs.back().second;
+        const int h = n / 2 / 32 * 32;
+        if (h < 128) break;
+        segs.back().second = h;
+        segs.emplace_back(t0 + h, n - h);
+    }
+    const int nseg = (int)segs.size();
     // device memory: per slot q, k, v, a, b, o for seg tokens of B sequences; the state;
     // A_log and dt_bias (each region 256-byte aligned)
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -129,7 +143,7 @@ cudaError_t launch_prefill_host(const FwdParams& hp, int seg, cudaStream_t strea
     if (e == cudaSuccess) e = cudaStreamWaitEvent(P.out, P.ev_comp[0], 0);
 
     for (int i = 0; i < nseg && e == cudaSuccess && *status == 0; ++i) {
-        const int s = i & 1, t0 = i * seg, n = (T - t0 < seg) ? T - t0 : seg;
+        const int s = i & 1, t0 = segs[i].first, n = segs[i].second;
         char* q = slot_ptr(s, 0);
         char* k = slot_ptr(s, bq);
         char* v = slot_ptr(s, 2 * bq);

@@ -201,7 +201,9 @@ GDR_API int gdr_prefill_chunked_cp(const void* q, const void* k, const void* v, 
  * asynchronously and overlap, pageable memory works but serialises them.
  *
  * The tokens are cut into chunk-aligned segments of seg_tokens (0: an eighth of T, at
- * least 256; otherwise a multiple of 32, else GDR_ERR_SHAPE).  Segment i's inputs are
+ * least 256; otherwise a multiple of 32, else GDR_ERR_SHAPE), the last one halved and
+ * its second half halved again (while the first parts keep at least 128 tokens), so that
+ * the final copy-out, which nothing overlaps, is short.  Segment i's inputs are
  * copied in on a library stream while segment i - 1 computes on `stream` and segment
  * i - 2's outputs are copied out on another library stream; each sequence's state stays
  * on the device between segments, so the result is the one-call result up to rounding

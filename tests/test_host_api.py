@@ -44,7 +44,9 @@ def _pinned(x, dtype):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("seg", [96, 0])
+# 96: ten full segments and a ragged one; 0: the default (256 here); 512: the last segment
+# cut in two, twice (512, 224, 128, 136 tokens)
+@pytest.mark.parametrize("seg", [96, 0, 512])
 def test_host_prefill_matches_oracle_and_device_call(seg):
     torch = pytest.importorskip("torch")
     B, T, Hk, Hv = 2, 1000, 2, 6  # 1000 = 10 segments of 96 + 40; ragged last chunk
