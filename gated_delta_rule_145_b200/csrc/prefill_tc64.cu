@@ -1113,8 +1113,9 @@ __device__ void o64_role(Sp64Smem& sm, const Sp64Ctx& x, int warp, int lane,
         ld_acc24s(tl + T_ACC1 + 96 * (s & 1) + j0, 0.f, o);
         warp_arrive64(&sm.acc1_free[s & 1], lane);
         // after G1(s + 1) was issued: the epilogue then overlaps the BD group's (other
-        // sub-partitions) rather than the S group's and the G1 issue
-        if (s + 1 < x.n && !w64(ab, &sm.g1_issued, (uint32_t)s & 1u)) break;
+        // sub-partitions) rather than the S group's and the G1 issue (erase = 0: the BD
+        // group runs ahead of the state, and P Delta(s) is read as soon as it is there)
+        if (!x.gla && s + 1 < x.n && !w64(ab, &sm.g1_issued, (uint32_t)s & 1u)) break;
         if (!w64(ab, &sm.acc4_full, (uint32_t)s & 1u)) break;
         tc_fence_after();
         ld_acc24s(tl + T_ACC4 + j0, e, o);
