@@ -45,7 +45,7 @@ struct SimtSmem {
     float KS[kC][kDVT];  // K S, then the right-hand side diag(beta)V - diag(beta e^G) K S
     float QS[kC][kDVT];
     float D[kC][kDVT];  // Delta
-    float beta[kC], G[kC], eG[kC], wC[kC];
+    float beta[kC], G[kC], Gl[kC], eG[kC], wC[kC];  // G as the pair G + Gl
 };
 
 template <int DK, typename Tin>
@@ -127,17 +127,15 @@ chunked_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
                 const size_t th = (size_t)(c0 + lane) * Hv + h;
                 gates(load1(a + th), load1(b + th), Al, dtb, g, beta);
             }
-            float G = g;  // inclusive scan over the chunk
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float x = __shfl_up_sync(0xffffffffu, G, o);
-                if (lane >= o) G += x;
-            }
+            float G, Gl;  // inclusive scan over the chunk, as a pair
+            scan32_pair(g, lane, G, Gl);
             const float GC = __shfl_sync(0xffffffffu, G, 31);
+            const float GCl = __shfl_sync(0xffffffffu, Gl, 31);
             sm.beta[lane] = beta;
             sm.G[lane] = G;
-            sm.eG[lane] = expf(G);
-            sm.wC[lane] = expf(GC - G);
+            sm.Gl[lane] = Gl;
+            sm.eG[lane] = expf(G + Gl);
+            sm.wC[lane] = expf((GC - G) + (GCl - Gl));
         }
         __syncthreads();
         // ---- Gram (K K^T, Q K^T) and K S, Q S: thread -> row i, 4 columns
@@ -159,11 +157,11 @@ chunked_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
                     qs[x] += qi * sdv[x];
                 }
             }
-            const float Gi = sm.G[i], bi = sm.beta[i];
+            const float Gi = sm.G[i], Gli = sm.Gl[i], bi = sm.beta[i];
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 const int j = j0 + x;
-                const float dec = j <= i ? expf(Gi - sm.G[j]) : 0.f;
+                const float dec = j <= i ? expf((Gi - sm.G[j]) + (Gli - sm.Gl[j])) : 0.f;
                 sm.A[i][j] = (erase && j < i) ? bi * dec * kk[x] : 0.f;  // erase = 0: A = 0
                 sm.P[i][j] = dec * qk[x];
                 sm.KS[i][j] = ks[x];

@@ -115,14 +115,7 @@ __device__ __forceinline__ void gates_fast64(float a, float b, float eA, float d
     beta = __frcp_rn(1.f + __expf(-b));
 }
 
-__device__ __forceinline__ float scan32(float x, int lane) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    return x;
-}
+constexpr float kLog2e = 1.4426950408889634f;
 
 // 2^x by the special-function unit (ex2.approx; results below the normal range flush to 0).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -182,9 +175,14 @@ struct alignas(1024) Prep64Smem {
         } w;
     };
     alignas(16) float beta[C64];
-    alignas(16) float G[C64];   // G of tokens 32-63 still lacks the first half's total
-    alignas(16) float G2[C64];  // the block's G times log2(e)
-    alignas(16) float G2r[C64]; // G2 - log2(r_k): a column's decay and key scale in one exponent
+    // G as a pair (gdr_common.cuh): the halves' scans (tokens 32-63 still lack the first
+    // half's total), then the block's G times log2(e) as Yh + Yl, and a column's lo part
+    // with its key scale folded in, Xl = Yl - log2(r_k)
+    alignas(16) float Gs[C64];
+    alignas(16) float Gsl[C64];
+    alignas(16) float Yh[C64];
+    alignas(16) float Yl[C64];
+    alignas(16) float Xl[C64];
     alignas(16) float rk[C64];
     alignas(16) float rq[C64];
     uint64_t bar_tma, bar_mma;
@@ -245,8 +243,20 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (i < n)
                 gates_fast64(__bfloat162float(ga), __bfloat162float(gb), expf(A_lg), dtb, g, bt);
             sm.beta[i] = bt;
-            sm.G[i] = scan32(g, lane);
+            float hi, lo;
+            scan32_pair(g, lane, hi, lo);
+            sm.Gs[i] = hi;
+            sm.Gsl[i] = lo;
         }
+    };
+    // token i's G times log2(e), as a pair (the product's rounding error by an fma)
+    auto g2pair = [&](int i, float& yh, float& yl) {
+        float hi = sm.Gs[i], lo = sm.Gsl[i];
+        if (i >= 32) pair_add(hi, lo, sm.Gs[31], sm.Gsl[31]);
+        const float ph = hi * kLog2e;
+        const float pl = fmaf(hi, kLog2e, -ph) + lo * kLog2e;
+        yh = ph + pl;
+        yl = pl - (yh - ph);
     };
     load_gates(h);
     if (tid == 0) {
@@ -287,7 +297,7 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ---- inverse norms of the K rows (0-63) and Q rows (64-127): a thread pair per row
     //      (the swizzle only permutes 16-byte pieces inside a row, which a sum ignores);
     //      with them the first value head's exponents (later heads: at the loop's top)
-    if (tid < C64) sm.G2[tid] = (sm.G[tid] + (tid >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f;
+    if (tid < C64) g2pair(tid, sm.Yh[tid], sm.Yl[tid]);
     if (ok) {
 #pragma unroll 1
         for (int e = 0; e < 2; ++e) {
@@ -298,8 +308,9 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (e == 0) {
                     const float r = rsqrtf(ss + kNormEps);
                     sm.rk[row] = r;
-                    sm.G2r[row] = (sm.G[row] + (row >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f -
-                                  __log2f(r);
+                    float yh, yl;
+                    g2pair(row, yh, yl);
+                    sm.Xl[row] = yl - __log2f(r);
                 } else {
                     sm.rq[row - 64] = rsqrtf(ss + kNormEps) * rsqrtf((float)DK);
                 }
@@ -321,17 +332,16 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncthreads();  // the previous head's last phase has read G and beta
             gates();
             __syncthreads();
-            // the block's G times log2(e), and with -log2(r_k): a column's decay and key
-            // scale in one exponent
+            // the block's G times log2(e) as a pair, and a column's lo part with -log2(r_k)
             if (tid < C64) {
-                const float g2 = (sm.G[tid] + (tid >= 32 ? sm.G[31] : 0.f)) * 1.4426950408889634f;
-                sm.G2[tid] = g2;
-                sm.G2r[tid] = g2 - __log2f(sm.rk[tid]);
+                float yh, yl;
+                g2pair(tid, yh, yl);
+                sm.Yh[tid] = yh;
+                sm.Yl[tid] = yl;
+                sm.Xl[tid] = yl - __log2f(sm.rk[tid]);
             }
             __syncthreads();
         }
-        const float G31 = sm.G[31];
-        auto Gf = [&](int j) { return sm.G[j] + (j >= 32 ? G31 : 0.f); };
 
         // ---- A rows into shared memory (warps 0, 1); P rows straight into the record's
         //      image rows 64-127 (warps 2, 3).  Accumulator row 32 w + lane (warps 0, 1: K K^T,
@@ -341,7 +351,7 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (erase || warp >= 2) {
             const bool arow = warp < 2;
             const int i = 32 * (warp & 1) + lane;
-            const float Gi2 = sm.G2[i];
+            const float Yhi = sm.Yh[i], Yli = sm.Yl[i];
             const float f = arow ? (erase ? sm.beta[i] * sm.rk[i] : 0.f) : sm.rq[i];
             // rows 0-31 (warps 0, 2) have nothing right of column 31: A there is never read and
             // the image's P chunks are written as zeros below
@@ -350,16 +360,21 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int kc = 0; kc < kc_end; ++kc) {
                 float v[8], p[8];
                 tmem_ld8(tmem + lane_base64(warp) + 8 * kc, v);
-                const float4 g0 = *reinterpret_cast<const float4*>(&sm.G2r[8 * kc]);
-                const float4 g1 = *reinterpret_cast<const float4*>(&sm.G2r[8 * kc + 4]);
-                const float gj[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                const float4 h0 = *reinterpret_cast<const float4*>(&sm.Yh[8 * kc]);
+                const float4 h1 = *reinterpret_cast<const float4*>(&sm.Yh[8 * kc + 4]);
+                const float4 l0 = *reinterpret_cast<const float4*>(&sm.Xl[8 * kc]);
+                const float4 l1 = *reinterpret_cast<const float4*>(&sm.Xl[8 * kc + 4]);
+                const float hj[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+                const float lj[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     const int jj = 8 * kc + e;
-                    // e^{G_i - G_j} r_k,j = 2^{G2_i - G2r_j}
-                    const float2 d = __ffma2_rn(make_float2(gj[e], gj[e + 1]), make_float2(-1.f, -1.f),
-                                                make_float2(Gi2, Gi2));
+                    // e^{G_i - G_j} r_k,j = 2^{(Yh_i - Yh_j) + (Yl_i - Xl_j)}
+                    const float2 m1 = make_float2(-1.f, -1.f);
+                    const float2 d = __fadd2_rn(
+                        __ffma2_rn(make_float2(hj[e], hj[e + 1]), m1, make_float2(Yhi, Yhi)),
+                        __ffma2_rn(make_float2(lj[e], lj[e + 1]), m1, make_float2(Yli, Yli)));
                     const float2 ex = make_float2(ex2_approx(d.x), ex2_approx(d.y));
                     const float2 pv = __fmul2_rn(__fmul2_rn(make_float2(f, f), ex),
                                                  make_float2(v[e], v[e + 1]));
@@ -537,12 +552,15 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (tid < C64) {
             const int i = tid;
             float* vec = reinterpret_cast<float*>(rc + r64::OFF_VEC);
-            const float Gi = Gf(i), GC = Gf(C64 - 1), eG = __expf(Gi);
+            // e^{G_i}, e^{G_C - G_i} and e^{G_C} as powers of two of the pairs
+            const float Yhi = sm.Yh[i], Yli = sm.Yl[i];
+            const float YhC = sm.Yh[C64 - 1], YlC = sm.Yl[C64 - 1];
+            const float eG = ex2_approx(Yhi + Yli);
             vec[r64::VEC_E + i] = eG * sm.rq[i];
-            vec[r64::VEC_D + i] = __expf(GC - Gi) * sm.rk[i];
+            vec[r64::VEC_D + i] = ex2_approx((YhC - Yhi) + (YlC - Yli)) * sm.rk[i];
             vec[r64::VEC_BETA + i] = sm.beta[i];
             vec[r64::VEC_W + i] = erase ? sm.beta[i] * eG * sm.rk[i] : 0.f;
-            if (i == 0) vec[r64::VEC_GAMMA] = __expf(GC);
+            if (i == 0) vec[r64::VEC_GAMMA] = ex2_approx(YhC + YlC);
         }
     }  // value heads of the key head
 }

@@ -116,6 +116,24 @@ def check_beta_zero_decay(lib):
     _close(o[0, :, 0], np.exp(G)[:, None] * (qh @ S0[0, 0]), 1e-12, "beta=0 outputs")
 
 
+def check_full_decay_keeps_only_the_last_write(lib):
+    """Saturated decay (a = +40, so each token's gamma is below e^-30): the state carries
+    only the current token's write, S_t = beta_t k_t v_t^T, so o_t = beta_t (q_t . k_t) v_t
+    and the final state is the last write, whatever S0 held."""
+    rng = np.random.default_rng(16)
+    dk, dv, T = 8, 6, 12
+    q, k, v, a, b, A_log, dtb, S0 = _rand_raw(rng, T, 1, 1, dk, dv, s0=1.0)
+    a[:] = 40.0
+    o, S = oracle.forward(q, k, v, a, b, A_log, dtb, S0, lib=lib)
+    qq, kk = q[0, :, 0].astype(np.float64), k[0, :, 0].astype(np.float64)
+    qh = qq / np.sqrt((qq * qq).sum(-1, keepdims=True) + 1e-6) / math.sqrt(dk)
+    kh = kk / np.sqrt((kk * kk).sum(-1, keepdims=True) + 1e-6)
+    beta = 1.0 / (1.0 + np.exp(-b[0, :, 0].astype(np.float64)))
+    vv = v[0, :, 0].astype(np.float64)
+    _close(o[0, :, 0], (beta * (qh * kh).sum(-1))[:, None] * vv, 1e-12, "full-decay outputs")
+    _close(S[0, 0], beta[-1] * np.outer(kh[-1], vv[-1]), 1e-12, "full-decay final state")
+
+
 def check_first_step(lib):
     """(vi) T = 1 from zero state with beta = 1/2, gamma = 1/2: S = k v^T / 2, o = (q.k) v / 2."""
     dk, dv = 4, 3
@@ -253,7 +271,8 @@ def check_grouped_heads_and_varlen(lib):
 
 
 PINS = [check_bruteforce, check_gla, check_chunk_invariance, check_beta_one_retrieval,
-        check_beta_zero_decay, check_first_step, check_orthogonal_keys, check_contraction,
+        check_beta_zero_decay, check_full_decay_keeps_only_the_last_write, check_first_step,
+        check_orthogonal_keys, check_contraction,
         check_streaming_equals_recompute, check_gate_values, check_normalisation_invariance,
         check_golden_hand_example, check_grouped_heads_and_varlen]
 
