@@ -17,7 +17,10 @@
  *   gdr_prefill_chunked*  -- the chunk-parallel UT-transform form (prefill);
  *   gdr_decode_step*      -- the sequential recurrence on a persistent state (decode);
  *   gdr_prefill_recurrent* -- the sequential recurrence over many tokens in one call.
- * They agree up to floating-point reassociation.  Inference only (no backward).
+ * They agree up to floating-point reassociation, for any gate values: the chunked form
+ * keeps each chunk's cumulative log-decay as a pair of floats, so its decay factors stay
+ * accurate where single tokens decay by hundreds of nats (gate inputs of +-40 are checked
+ * against an fp64 reference).  Inference only (no backward).
  * The "_f32" suffix marks fp32 q, k, v, a, b (tessera PR #77 names its C-ABI symbols
  * the same way); the unsuffixed calls take bf16 q, k, v, a, b.
  *
@@ -36,6 +39,8 @@
  *     abort; they return one of the GDR_* codes below.  GDR_ERR_CUDA reports a launch
  *     error taken from cudaGetLastError (which clears it).
  *   - Supported head sizes: dk == dv in {32, 64, 128}; chunk == 32.
+ *   - Sizes: every device offset is 64-bit, so tensors may exceed 2^31 elements; token
+ *     counts (T, or the packed total with cu_seqlens) and B are int.
  *   - Memory: the bf16 chunked prefill at dk = dv = 128 needs a workspace of
  *     33808 bytes per (64-token block, value head) -- 208 MB for T = 8192, Hv = 48 -- which the
  *     library takes, per call, from a private stream-ordered pool of the current device
