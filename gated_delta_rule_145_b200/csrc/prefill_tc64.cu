@@ -329,7 +329,7 @@ intra64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int gi = 0; gi < grp; ++gi, ++h) {
         uint8_t* rc = ws + ((size_t)f * Hv + h) * r64::BYTES;
         if (gi > 0) {
-            __syncthreads();  // the previous head's last phase has read G and beta
+            __syncthreads();  // the previous head's last phase has read its exponents and beta
             gates();
             __syncthreads();
             // the block's G times log2(e) as a pair, and a column's lo part with -log2(r_k)
