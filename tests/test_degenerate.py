@@ -118,3 +118,32 @@ def test_decode_degenerate(case):
     ro, rS = oracle_forward(inp)
     assert_parity(o, ro, TAU["bf16"], f"{case} decode o")
     assert_parity(_np(state), rS, TAU["bf16"], f"{case} decode state")
+
+
+@pytest.mark.parametrize("case", ["full_decay", "mixed_gates", "beta_one"])
+@pytest.mark.parametrize("d", [32, 64])
+def test_prefill_degenerate_small_heads(case, d):
+    """the CUDA-core chunked kernel with bf16 inputs (head sizes below 128)"""
+    inp = degenerate_inputs(case, d=d)
+    o, S = _prefill(inp, "chunked")
+    ro, rS = oracle_forward(inp)
+    assert_parity(o, ro, TAU["bf16"], f"{case} d={d} o")
+    assert_parity(S, rS, TAU["bf16"], f"{case} d={d} final state")
+
+
+@pytest.mark.parametrize("case", ["full_decay", "mixed_gates", "no_decay"])
+def test_context_parallel_degenerate(case):
+    """one sequence in three segments: segment maps, their composition, then the prefill
+    from the composed start states"""
+    inp = degenerate_inputs(case, B=1, T=333)
+    d = to_device(inp)
+    out = torch.empty((1, 333, 4, 128), device="cuda")
+    fin = torch.empty((1, 4, 128, 128), device="cuda")
+    gdr.gdr_prefill_chunked_cp(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"],
+                               d["dt_bias"], d["init_state"], out, fin, 333, 2, 4, 128, 128,
+                               32, 3)
+    torch.cuda.synchronize()
+    assert gdr.gdr_device_status() == gdr.GDR_OK
+    ro, rS = oracle_forward(inp)
+    assert_parity(_np(out), ro, TAU["bf16"], f"{case} context-parallel o")
+    assert_parity(_np(fin), rS, TAU["bf16"], f"{case} context-parallel final state")
